@@ -1,0 +1,449 @@
+"""Benchmark of the chunk-causal 3D-RoPE attention path on B200.
+
+One step = one DiT-layer attention call (dz_chunk_attn_forward) on the
+single-layer inference workload: B=1, 40 heads, head_dim 128, a 464-token noisy
+chunk (2 latent frames of 11x20 tokens + 24 action tokens) over a KV cache of 4
+clean chunks plus itself (2320 keys).  The call fuses the token metadata, the
+3D rotary of q and of the chunk's own k, the tile classification, QK^T, the
+online softmax, PV and the split-KV combine.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line on rank 0.  Timing: K calls replayed from CUDA graphs
+that cycle through enough distinct input sets to exceed the 126 MB L2, timed
+with CUDA events on the launching stream between barriers + synchronize, max
+over ranks.  ``--impl reference`` times the CPU fp64 oracle instead (bounded
+samples of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from causal_video_diffusion_rope_b200 import synth  # noqa: E402
+
+METRIC = ("chunk-causal attn TFLOP/s and % of B200 BF16 peak; "
+          "µs per DiT-layer attention call")
+WORKLOAD = synth.WORKLOADS[1]
+L2_BYTES = 126 * 1024 * 1024
+KERNEL_SOURCES = ["causal_video_diffusion_rope_b200/csrc/dz_attn.cu",
+                  "causal_video_diffusion_rope_b200/csrc/dz_internal.cuh",
+                  "causal_video_diffusion_rope_b200/csrc/dz_ptx.cuh"]
+
+
+def visible_pairs(w: synth.Workload) -> int:
+    """Visible (query, key) pairs of one batch item and head of a call (chunk rule)."""
+    lay = w.layout
+    L = lay.chunk_len
+    if lay.mode == synth.MODE_DECODE:
+        return L * (w.cache_tokens + L)
+    if lay.mode == synth.MODE_CROSS:
+        return lay.q_len * lay.kv_len
+    if lay.mode == synth.MODE_PREFILL:
+        return sum(L * (c + 1) * L for c in range(lay.num_chunks))
+    N = lay.num_chunks
+    clean = sum(L * (i + 1) * L for i in range(N))
+    noisy = sum(L * (i * L + L) for i in range(N))
+    return clean + noisy
+
+
+def step_flops(w: synth.Workload) -> float:
+    """Algorithmic FLOPs of one call: 4 * head_dim per visible pair per head per batch item."""
+    return 4.0 * w.head_dim * visible_pairs(w) * w.heads * w.layout.batch
+
+
+def step_bytes(w: synth.Workload) -> float:
+    """Bytes one call must move at least once: q, k, v, cached K/V, out (bf16)."""
+    lay = w.layout
+    row = w.heads * w.head_dim * 2 * lay.batch
+    return row * (3 * lay.q_len + 2 * w.cache_tokens + lay.q_len)
+
+
+def sources_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops", 1590.0), d.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+def ncu_traffic():
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary,
+    or None if it was taken on different kernel sources."""
+    path = os.path.join(ROOT, "profiles", "attn_decode_b1_h40_q464_cache4.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("sources_hash") != sources_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.t_on = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------------- CPU legs
+
+def oracle_rate(w: synth.Workload, inp, rng, budget_s: float, rows_per_call: int):
+    """Time the fp64 oracle on sampled query rows of workload ``w`` until ``budget_s`` passes.
+
+    Returns (TFLOP/s, calls, seconds); FLOPs are counted like the GPU's (4*D per visible pair).
+    """
+    from oracle import dz_oracle as O
+    lay = w.layout
+    keys = w.cache_tokens + lay.chunk_len
+    flops = 0.0
+    calls = 0
+    t0 = time.perf_counter()
+    while True:
+        rows = [(int(rng.integers(lay.batch)), int(rng.integers(lay.q_len)),
+                 int(rng.integers(w.heads))) for _ in range(rows_per_call)]
+        O.attention_rows(inp["q"], inp["k"], inp["v"], rows, lay.mode, lay.frames_per_chunk,
+                         lay.grid_h, lay.grid_w, lay.n_action, lay.num_chunks,
+                         t_offset=lay.t_offset, cache_k_bits=inp["cache_k"],
+                         cache_v_bits=inp["cache_v"], cache_len=w.cache_tokens)
+        flops += 4.0 * w.head_dim * keys * rows_per_call
+        calls += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return flops / dt / 1e12, calls, dt
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_full_call_rate(w: synth.Workload, budget_s: float):
+    """The oracle computing whole calls of ``w`` (all heads) for about ``budget_s``."""
+    from oracle import dz_oracle as O
+    lay = w.layout
+    inp = synth.make_inputs(w, 0)
+    t0 = time.perf_counter()
+    n = 0
+    heads_done = 0
+    # whole calls if they fit the budget, else head slices of one call
+    while time.perf_counter() - t0 < budget_s:
+        h = heads_done % w.heads
+        O.chunk_attn_forward(inp["q"], inp["k"], inp["v"], lay.mode, lay.frames_per_chunk,
+                             lay.grid_h, lay.grid_w, lay.n_action, lay.num_chunks,
+                             t_offset=lay.t_offset, cache_k_bits=inp["cache_k"],
+                             cache_v_bits=inp["cache_v"], cache_len=w.cache_tokens,
+                             heads=slice(h, h + 4))
+        heads_done += 4
+        n += 1
+    dt = time.perf_counter() - t0
+    flops = step_flops(w) / w.heads * heads_done
+    return flops / dt / 1e12, heads_done, dt
+
+
+# ----------------------------------------------------------------------------------- GPU leg
+
+def run_gpu(args, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    from causal_video_diffusion_rope_b200 import dz
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOAD
+    lay = w.layout
+    B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
+    per_set = step_bytes(w)
+    n_sets = max(2, int(math.ceil(3 * L2_BYTES / per_set)))
+    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len))
+    dl = dz.layout_from(lay)
+    sets = []
+    for i in range(n_sets):
+        inp = synth.make_inputs(w, 1000 * rank + i)
+        s = {k: torch.from_numpy(inp[k].view(np.int16)).to(dev).view(torch.bfloat16)
+             for k in ("q", "k", "v", "cache_k", "cache_v")}
+        s["out"] = torch.empty((B, L, H, D), dtype=torch.bfloat16, device=dev)
+        s["cache"] = dz.make_cache(s["cache_k"], s["cache_v"], B, w.cache_tokens,
+                                   w.cache_tokens, L)
+        sets.append(s)
+    stream = torch.cuda.Stream(device=dev)
+
+    def call(i):
+        s = sets[i % n_sets]
+        dz.dz_chunk_attn_forward(h, s["q"], s["k"], s["v"], s["cache"], dl, s["out"], stream)
+
+    # warm-up outside any graph
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            call(i)
+    stream.synchronize()
+    dz.dz_attn_sync_status(h, stream)
+
+    # graphs of g calls cycling through the input sets
+    g = n_sets * max(1, 240 // n_sets)
+    graphs = {}
+
+    def graph_of(n):
+        if n not in graphs:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for i in range(n):
+                    call(i)
+            graphs[n] = gr
+        return graphs[n]
+
+    full, rem = divmod(args.steps, g)
+    if full:
+        graph_of(g)
+    if rem:
+        graph_of(rem)
+    # warm the graphs once
+    with torch.cuda.stream(stream):
+        if full:
+            graphs[g].replay()
+        if rem:
+            graphs[rem].replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(full):
+            graphs[g].replay()
+        if rem:
+            graphs[rem].replay()
+        e1.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1)
+    dz.dz_attn_sync_status(h, stream)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    flops = step_flops(w)
+    tflops_total = flops * args.steps * world / (ms * 1e-3) / 1e12
+
+    # ---- end to end: host buffers in, result out, through the same C-ABI call
+    e2e = None
+    s0 = sets[0]
+    hq = torch.empty_like(s0["q"], device="cpu").pin_memory()
+    hk = torch.empty_like(s0["k"], device="cpu").pin_memory()
+    hv = torch.empty_like(s0["v"], device="cpu").pin_memory()
+    ho = torch.empty_like(s0["out"], device="cpu").pin_memory()
+    hq.copy_(s0["q"].cpu())
+    hk.copy_(s0["k"].cpu())
+    hv.copy_(s0["v"].cpu())
+    dq, dk, dv = torch.empty_like(s0["q"]), torch.empty_like(s0["k"]), torch.empty_like(s0["v"])
+    n_e2e = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        dz.dz_chunk_attn_forward(h, dq, dk, dv, s0["cache"], dl, s0["out"], stream)
+        ho.copy_(s0["out"], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            e2e_step()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        x0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        x1.record(stream)
+    stream.synchronize()
+    ems = x0.elapsed_time(x1)
+    if world > 1:
+        t = torch.tensor([ems], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ems = float(t.item())
+    dz.dz_attn_sync_status(h, stream)
+    e2e = {"value": round(flops * n_e2e * world / (ems * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(hq.numel() * 2 * 3), "d2h_bytes_per_step": int(ho.numel() * 2),
+           "ms_per_step": round(ems / n_e2e, 4), "steps": n_e2e}
+
+    for gr in graphs.values():
+        del gr
+    graphs.clear()
+    dz.dz_attn_destroy(h)
+    return ms_per_step, tflops_total, clocks, e2e
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=48000)
+    ap.add_argument("--warmup", type=int, default=240)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0,
+                    help="seconds of oracle CPU work for the cpu_baseline field")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    w = WORKLOAD
+    config = {"workload": w.name, "batch": w.layout.batch, "heads": w.heads,
+              "head_dim": w.head_dim, "q_tokens": w.layout.q_len,
+              "keys": w.cache_tokens + w.layout.chunk_len, "cache_tokens": w.cache_tokens,
+              "mode": "decode", "rope": "3d t/h/w 22/21/21 base 1e4 fused",
+              "flop_per_step": step_flops(w)}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        budget = 150.0 / (args.steps + args.warmup)
+        # each step: the oracle on a bounded sample of query rows of the same call
+        rows_per_step = 1
+        rate = []
+        t_all = time.perf_counter()
+        inp = synth.make_inputs(w, 0)
+        rng = np.random.default_rng(0)
+        for i in range(args.warmup + args.steps):
+            r, calls, dt = oracle_rate(w, inp, rng, budget, rows_per_step)
+            if i >= args.warmup:
+                rate.append((r, dt))
+        elapsed = sum(dt for _, dt in rate)
+        value = float(np.mean([r for r, _ in rate]))
+        cores = blas_threads()
+        line = {"impl": "reference", "metric": METRIC, "value": round(value, 6),
+                "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / max(1, len(rate)), 3),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": dict(config, l2="n/a (CPU)"),
+                "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
+                                 "kind": "oracle",
+                                 "sample": f"{rows_per_step} query row(s) of the call per step, "
+                                           f"~{budget * 1e3:.1f} ms of oracle work per step"},
+                "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "wall_s": round(time.perf_counter() - t_all, 1)}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    cpu = None
+    if rank == 0:
+        # the oracle, timed on this host's cores before the GPU work starts
+        r, heads_done, dt = oracle_full_call_rate(w, args.cpu_budget)
+        cpu = {"value": round(r, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+               "kind": "oracle",
+               "sample": f"{heads_done} of {w.heads} heads of the call (4-head slices), "
+                         f"{dt:.1f} s of fp64 oracle work"}
+    ms_per_step, tflops, clocks, e2e = run_gpu(args, rank, world, local_rank)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak_tf, peak_hbm, peak_kind = measured_peaks()
+    per_gpu_tf = step_flops(w) / (ms_per_step * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": round(per_gpu_tf, 2), "peak": peak_tf,
+            "unit": "TFLOP/s", "frac": round(per_gpu_tf / peak_tf, 4),
+            "traffic": ncu_traffic(), "peak_kind": f"{peak_kind} bf16 (burst)",
+            "kernel": "chunk_attn_kernel",
+            "hbm_frac": round(step_bytes(w) / (ms_per_step * 1e-3) / 1e9 / peak_hbm, 4)}
+    n_sets = max(2, int(math.ceil(3 * L2_BYTES / step_bytes(w))))
+    line = {"metric": METRIC, "value": round(tflops, 3), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6), "us_per_call": round(ms_per_step * 1e3, 3),
+            "pct_of_bf16_peak": round(100 * per_gpu_tf / peak_tf, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(config, l2=f"inputs cycle through {n_sets} sets "
+                                      f"({n_sets * step_bytes(w) / 2**20:.0f} MiB > 126 MB L2)",
+                           parallelism=f"dp{world} (independent replicas of the call)"),
+            "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,383 @@
+// Host side of the C ABI declared in include/dz.h: argument checks, rotary
+// tables, TMA tensor maps, the work split and the kernel launches.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/dz.h"
+#include "dz_internal.cuh"
+
+struct dz_attn {
+  int device;
+  int num_sms;
+  dz_attn_desc desc;
+  float2* rope_tab;
+  int off_t, off_h, off_w;
+  float* ws;           // 2 partial slots per CTA of the persistent grid
+  int* counters;       // one per (batch, head, query group, Q tile)
+  size_t n_counters;
+  int* status;         // device status word
+  PFN_cuTensorMapEncodeTiled_v12000 encode;
+};
+
+namespace {
+
+using dz::cdiv;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// With DZ_DEBUG set in the environment, failing CUDA calls are reported on stderr.
+bool debug_on() {
+  static const bool on = std::getenv("DZ_DEBUG") != nullptr;
+  return on;
+}
+
+dz_status cuda_status(cudaError_t e, const char* where = "") {
+  if (e == cudaSuccess) return DZ_OK;
+  if (debug_on()) std::fprintf(stderr, "[dz] %s: %s\n", where, cudaGetErrorString(e));
+  return DZ_ERR_CUDA;
+}
+
+// 4-D view [B][rows][H][128] of a bf16 BSHD buffer whose batch stride is
+// `rows_alloc` tokens; 64 x 1 x 128 x 1 boxes with 128-byte swizzle.
+dz_status make_map(const dz_attn* a, CUtensorMap* m, const void* base, int B, int rows,
+                   int rows_alloc, int H) {
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(dz::HEAD_DIM), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(B)};
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(H) * dz::HEAD_DIM * 2;
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(dz::HEAD_DIM) * 2, row_bytes,
+                                 row_bytes * static_cast<cuuint64_t>(rows_alloc)};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(dz::TILE_N), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = a->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && debug_on())
+    std::fprintf(stderr, "[dz] cuTensorMapEncodeTiled failed (%d): dims %llu %llu %llu %llu\n",
+                 static_cast<int>(r), static_cast<unsigned long long>(dims[0]),
+                 static_cast<unsigned long long>(dims[1]), static_cast<unsigned long long>(dims[2]),
+                 static_cast<unsigned long long>(dims[3]));
+  return r == CUDA_SUCCESS ? DZ_OK : DZ_ERR_CUDA;
+}
+
+dz_status check_geom(const dz_chunk_layout* l) {
+  if (l->frames_per_chunk < 1 || l->grid_h < 1 || l->grid_w < 1 || l->n_action < 0 ||
+      l->t_offset < 0 || l->num_chunks < 0 || l->batch < 1)
+    return DZ_ERR_INVALID_ARG;
+  const long long L = static_cast<long long>(l->frames_per_chunk) * l->grid_h * l->grid_w +
+                      l->n_action;
+  if (L > (1 << 24)) return DZ_ERR_SHAPE;
+  return DZ_OK;
+}
+
+dz::ChunkGeom geom_of(const dz_chunk_layout* l) {
+  dz::ChunkGeom g;
+  g.F = l->frames_per_chunk;
+  g.gh = l->grid_h;
+  g.gw = l->grid_w;
+  g.L = l->frames_per_chunk * l->grid_h * l->grid_w + l->n_action;
+  g.t_offset = l->t_offset;
+  return g;
+}
+
+dz::RopeTables tables_of(const dz_attn* a) {
+  dz::RopeTables r;
+  r.tab = a->rope_tab;
+  r.off_t = a->off_t;
+  r.off_h = a->off_h;
+  r.off_w = a->off_w;
+  r.pt = a->desc.rope_pairs_t;
+  r.ph = a->desc.rope_pairs_h;
+  r.pw = a->desc.rope_pairs_w;
+  return r;
+}
+
+// Chunks [first, last] of `g` must lie inside the rotary tables.
+dz_status check_positions(const dz_attn* a, const dz::ChunkGeom& g, long long first_chunk,
+                          long long last_chunk) {
+  if (last_chunk < first_chunk) return DZ_OK;
+  const long long t_max = g.t_offset + last_chunk * g.F + g.F - 1;
+  if (t_max >= a->desc.max_pos_t || g.gh > a->desc.max_pos_h || g.gw > a->desc.max_pos_w)
+    return DZ_ERR_SHAPE;
+  return DZ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dz_status_string(dz_status s) {
+  switch (s) {
+    case DZ_OK: return "ok";
+    case DZ_ERR_INVALID_ARG: return "invalid argument";
+    case DZ_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case DZ_ERR_SHAPE: return "unsupported shape";
+    case DZ_ERR_CAPACITY: return "capacity exceeded";
+    case DZ_ERR_CUDA: return "CUDA error";
+    case DZ_ERR_UNSUPPORTED: return "unsupported";
+    case DZ_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+dz_status dz_attn_create(dz_attn_t* out, const dz_attn_desc* d) {
+  if (!out || !d) return DZ_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (d->head_dim != dz::HEAD_DIM) return DZ_ERR_SHAPE;
+  if (d->num_heads < 1 || d->num_heads > 256) return DZ_ERR_SHAPE;
+  if (d->rope_pairs_t < 0 || d->rope_pairs_h < 0 || d->rope_pairs_w < 0 ||
+      d->rope_pairs_t + d->rope_pairs_h + d->rope_pairs_w != dz::HEAD_DIM / 2)
+    return DZ_ERR_SHAPE;
+  if (!(d->rope_base > 1.0) || !std::isfinite(d->rope_base)) return DZ_ERR_SHAPE;
+  if (d->max_batch < 1 || d->max_q_tokens < 1 || d->max_pos_t < 1 || d->max_pos_h < 1 ||
+      d->max_pos_w < 1)
+    return DZ_ERR_SHAPE;
+  if (cdiv(d->max_q_tokens, dz::Q_GROUP) > dz::MAX_Q_GROUPS) return DZ_ERR_CAPACITY;
+  if (static_cast<long long>(d->max_pos_t) * d->rope_pairs_t +
+          static_cast<long long>(d->max_pos_h) * d->rope_pairs_h +
+          static_cast<long long>(d->max_pos_w) * d->rope_pairs_w > (1ll << 28))
+    return DZ_ERR_CAPACITY;
+
+  dz_attn* a = new (std::nothrow) dz_attn();
+  if (!a) return DZ_ERR_CUDA;
+  a->desc = *d;
+  if (cudaGetDevice(&a->device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&a->num_sms, cudaDevAttrMultiProcessorCount, a->device) !=
+          cudaSuccess) {
+    delete a;
+    return DZ_ERR_CUDA;
+  }
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+          cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn) {
+    delete a;
+    return DZ_ERR_CUDA;
+  }
+  a->encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+
+  // rotary tables, built in double and stored as float (cos, sin)
+  const int pt = d->rope_pairs_t, ph = d->rope_pairs_h, pw = d->rope_pairs_w;
+  a->off_t = 0;
+  a->off_h = d->max_pos_t * pt;
+  a->off_w = a->off_h + d->max_pos_h * ph;
+  const size_t n_tab = static_cast<size_t>(a->off_w) + static_cast<size_t>(d->max_pos_w) * pw;
+  std::vector<float2> tab(n_tab > 0 ? n_tab : 1);
+  auto fill = [&](int off, int npos, int npairs) {
+    for (int j = 0; j < npairs; ++j) {
+      const double omega = std::pow(d->rope_base, -2.0 * j / (2.0 * npairs));
+      for (int p = 0; p < npos; ++p) {
+        const double th = static_cast<double>(p) * omega;
+        tab[off + static_cast<size_t>(p) * npairs + j] =
+            make_float2(static_cast<float>(std::cos(th)), static_cast<float>(std::sin(th)));
+      }
+    }
+  };
+  fill(a->off_t, d->max_pos_t, pt);
+  fill(a->off_h, d->max_pos_h, ph);
+  fill(a->off_w, d->max_pos_w, pw);
+
+  const int n_qg_max = cdiv(d->max_q_tokens, dz::Q_GROUP);
+  a->n_counters = static_cast<size_t>(d->max_batch) * d->num_heads * n_qg_max * dz::Q_TILES;
+  const size_t ws_floats = 2ull * a->num_sms * dz::PART_FLOATS;
+  cudaError_t e = cudaMalloc(&a->rope_tab, tab.size() * sizeof(float2));
+  if (e == cudaSuccess) e = cudaMalloc(&a->ws, ws_floats * sizeof(float));
+  if (e == cudaSuccess) e = cudaMalloc(&a->counters, a->n_counters * sizeof(int));
+  if (e == cudaSuccess) e = cudaMalloc(&a->status, sizeof(int));
+  if (e == cudaSuccess)
+    e = cudaMemcpy(a->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaMemset(a->counters, 0, a->n_counters * sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(a->status, 0, sizeof(int));
+  if (e != cudaSuccess) {
+    cudaFree(a->rope_tab);
+    cudaFree(a->ws);
+    cudaFree(a->counters);
+    cudaFree(a->status);
+    delete a;
+    return DZ_ERR_CUDA;
+  }
+  *out = a;
+  return DZ_OK;
+}
+
+dz_status dz_attn_destroy(dz_attn_t a) {
+  if (!a) return DZ_ERR_INVALID_ARG;
+  cudaError_t e = cudaDeviceSynchronize();
+  cudaFree(a->rope_tab);
+  cudaFree(a->ws);
+  cudaFree(a->counters);
+  cudaFree(a->status);
+  delete a;
+  return cuda_status(e);
+}
+
+dz_status dz_rope3d(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
+                    const dz_chunk_layout* layout, int32_t first_chunk, void* stream) {
+  if (!a || !x || !y || !layout || B < 1 || S < 0 || first_chunk < 0) return DZ_ERR_INVALID_ARG;
+  dz_chunk_layout l = *layout;
+  l.batch = B;
+  l.num_chunks = 0;
+  dz_status st = check_geom(&l);
+  if (st != DZ_OK) return st;
+  if (!aligned16(x) || !aligned16(y)) return DZ_ERR_ALIGNMENT;
+  if (S == 0) return DZ_OK;
+  const dz::ChunkGeom g = geom_of(&l);
+  st = check_positions(a, g, first_chunk, first_chunk + (S - 1) / g.L);
+  if (st != DZ_OK) return st;
+  return cuda_status(dz::launch_rope3d(x, y, B, S, a->desc.num_heads, g, first_chunk,
+                                       tables_of(a), static_cast<cudaStream_t>(stream)),
+                     "rope3d launch");
+}
+
+dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const void* v,
+                                const dz_kvcache* cache, const dz_chunk_layout* l, void* out,
+                                void* stream) {
+  if (!a || !q || !k || !v || !l || !out) return DZ_ERR_INVALID_ARG;
+  if (l->mode < DZ_MODE_DECODE || l->mode > DZ_MODE_CROSS) return DZ_ERR_INVALID_ARG;
+  dz_status st = check_geom(l);
+  if (st != DZ_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return DZ_ERR_ALIGNMENT;
+  if (l->batch > a->desc.max_batch) return DZ_ERR_CAPACITY;
+  const int H = a->desc.num_heads;
+  const dz::ChunkGeom g = geom_of(l);
+  const long long L = g.L;
+  long long Sq = 0, Sk = 0;
+  int cache_len = 0;
+  switch (l->mode) {
+    case DZ_MODE_DECODE:
+      Sq = Sk = L;
+      if (cache) {
+        if (!cache->k || !cache->v) return DZ_ERR_INVALID_ARG;
+        if (!aligned16(cache->k) || !aligned16(cache->v)) return DZ_ERR_ALIGNMENT;
+        if (cache->batch != l->batch || cache->len_tokens < 0 ||
+            cache->len_tokens > cache->capacity_tokens)
+          return DZ_ERR_INVALID_ARG;
+        cache_len = cache->len_tokens;
+      }
+      break;
+    case DZ_MODE_TEACHER_FORCING:
+      if (cache) return DZ_ERR_INVALID_ARG;
+      if (l->num_chunks < 1) return DZ_ERR_INVALID_ARG;
+      Sq = Sk = 2 * L * l->num_chunks;
+      break;
+    case DZ_MODE_PREFILL:
+      if (cache) return DZ_ERR_INVALID_ARG;
+      if (l->num_chunks < 1) return DZ_ERR_INVALID_ARG;
+      Sq = Sk = L * l->num_chunks;
+      break;
+    case DZ_MODE_CROSS:
+      if (cache) return DZ_ERR_INVALID_ARG;
+      if (l->num_chunks < 1 || l->kv_len < 1) return DZ_ERR_INVALID_ARG;
+      Sq = L * l->num_chunks;
+      Sk = l->kv_len;
+      break;
+  }
+  if (Sq > a->desc.max_q_tokens) return DZ_ERR_CAPACITY;
+  if (Sk > (1 << 28) || static_cast<long long>(cache_len) + Sk > (1 << 28)) return DZ_ERR_SHAPE;
+  if (l->mode == DZ_MODE_DECODE) {
+    st = check_positions(a, g, l->num_chunks, l->num_chunks);
+  } else if (l->mode != DZ_MODE_CROSS) {
+    st = check_positions(a, g, 0, l->num_chunks - 1);
+  }
+  if (st != DZ_OK) return st;
+
+  dz::AttnLaunch p;
+  std::memset(&p, 0, sizeof(p));
+  p.sched.mode = l->mode;
+  p.sched.Sq = static_cast<int>(Sq);
+  p.sched.Sk = static_cast<int>(Sk);
+  p.sched.L = static_cast<int>(L);
+  p.sched.N = l->num_chunks;
+  p.sched.cache_len = cache_len;
+  p.sched.nkc = cdiv(cache_len, dz::TILE_N);
+  p.sched.nks = cdiv(static_cast<int>(Sk), dz::TILE_N);
+  p.n_qg = cdiv(static_cast<int>(Sq), dz::Q_GROUP);
+  if (p.n_qg > dz::MAX_Q_GROUPS) return DZ_ERR_CAPACITY;
+  long long per_bh = 0;
+  for (int qg = 0; qg < p.n_qg; ++qg) per_bh += dz::unit_tile_count(p.sched, qg);
+  p.W = per_bh * l->batch * H;
+  if (p.W <= 0) return DZ_ERR_SHAPE;
+  p.grid = static_cast<int>(p.W < a->num_sms ? p.W : a->num_sms);
+  p.B = l->batch;
+  p.H = H;
+  p.geom = g;
+  p.rope = tables_of(a);
+  p.rope_q = p.rope_k = (l->mode != DZ_MODE_CROSS) ? 1 : 0;
+  p.out = out;
+  p.ws = a->ws;
+  p.counters = a->counters;
+  p.status = a->status;
+
+  st = make_map(a, &p.tm_q, q, l->batch, static_cast<int>(Sq), static_cast<int>(Sq), H);
+  if (st == DZ_OK) st = make_map(a, &p.tm_k, k, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
+  if (st == DZ_OK) st = make_map(a, &p.tm_v, v, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
+  if (st == DZ_OK && cache_len > 0) {
+    st = make_map(a, &p.tm_ck, cache->k, l->batch, cache_len, cache->capacity_tokens, H);
+    if (st == DZ_OK)
+      st = make_map(a, &p.tm_cv, cache->v, l->batch, cache_len, cache->capacity_tokens, H);
+  }
+  if (st != DZ_OK) return st;
+  return cuda_status(dz::launch_attention(p, static_cast<cudaStream_t>(stream)),
+                     "attention launch");
+}
+
+dz_status dz_kvcache_append(dz_attn_t a, dz_kvcache* c, const void* k, const void* v,
+                            void* stream) {
+  if (!a || !c || !k || !v || !c->k || !c->v) return DZ_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->chunk_len < 1 || c->len_tokens < 0 || c->capacity_tokens < 0 ||
+      c->len_tokens > c->capacity_tokens)
+    return DZ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(c->k) || !aligned16(c->v))
+    return DZ_ERR_ALIGNMENT;
+  if (static_cast<long long>(c->len_tokens) + c->chunk_len > c->capacity_tokens)
+    return DZ_ERR_CAPACITY;
+  cudaError_t e = dz::launch_kv_copy(k, v, c->k, c->v, c->batch, c->chunk_len, a->desc.num_heads,
+                                     c->capacity_tokens, c->len_tokens,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return DZ_ERR_CUDA;
+  c->len_tokens += c->chunk_len;
+  return DZ_OK;
+}
+
+dz_status dz_kvcache_replace(dz_attn_t a, dz_kvcache* c, int32_t chunk_index, const void* k,
+                             const void* v, void* stream) {
+  if (!a || !c || !k || !v || !c->k || !c->v) return DZ_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->chunk_len < 1 || c->len_tokens < 0 ||
+      c->len_tokens > c->capacity_tokens || chunk_index < 0)
+    return DZ_ERR_INVALID_ARG;
+  if (static_cast<long long>(chunk_index + 1) * c->chunk_len > c->len_tokens)
+    return DZ_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(c->k) || !aligned16(c->v))
+    return DZ_ERR_ALIGNMENT;
+  return cuda_status(dz::launch_kv_copy(k, v, c->k, c->v, c->batch, c->chunk_len,
+                                        a->desc.num_heads, c->capacity_tokens,
+                                        chunk_index * c->chunk_len,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+dz_status dz_attn_sync_status(dz_attn_t a, void* stream) {
+  if (!a) return DZ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DZ_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpy(&word, a->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DZ_ERR_CUDA;
+  if (word != 0) {
+    // a kernel gave up mid-call: clear the word and the split counters it may have left
+    if (cudaMemset(a->status, 0, sizeof(int)) != cudaSuccess ||
+        cudaMemset(a->counters, 0, a->n_counters * sizeof(int)) != cudaSuccess ||
+        cudaDeviceSynchronize() != cudaSuccess)
+      return DZ_ERR_CUDA;
+    return DZ_ERR_TIMEOUT;
+  }
+  return DZ_OK;
+}
+
+}  // extern "C"

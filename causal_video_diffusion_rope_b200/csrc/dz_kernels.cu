@@ -1,0 +1,86 @@
+// Bandwidth-bound kernels: KV-cache append/replace (a 16-byte vectorised
+// copy) and the standalone 3D rotary embedding.
+#include "dz_internal.cuh"
+#include "dz_ptx.cuh"
+
+namespace dz {
+
+// ---------------------------------------------------------------------------
+// KV-cache chunk copy.  One chunk of keys and values, bf16 [B][rows][H][128],
+// is contiguous per batch item; in the cache [B][cap][H][128] it lands at rows
+// [dst_row0, dst_row0 + rows).  blockIdx.y selects (tensor, batch item); each
+// thread moves 4 independent 16-byte vectors per iteration (grid-stride).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) kv_copy_kernel(const uint4* __restrict__ k,
+                                                      const uint4* __restrict__ v,
+                                                      uint4* __restrict__ ck,
+                                                      uint4* __restrict__ cv, int B,
+                                                      long long span_vecs, long long src_stride,
+                                                      long long dst_stride, long long dst_off) {
+  const int which = blockIdx.y / B;  // 0 = keys, 1 = values
+  const int b = blockIdx.y - which * B;
+  const uint4* src = (which == 0 ? k : v) + static_cast<long long>(b) * src_stride;
+  uint4* dst = (which == 0 ? ck : cv) + static_cast<long long>(b) * dst_stride + dst_off;
+  const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
+  long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * step < span_vecs; i += 4 * step) {
+    const uint4 a0 = src[i], a1 = src[i + step], a2 = src[i + 2 * step], a3 = src[i + 3 * step];
+    dst[i] = a0;
+    dst[i + step] = a1;
+    dst[i + 2 * step] = a2;
+    dst[i + 3 * step] = a3;
+  }
+  for (; i < span_vecs; i += step) dst[i] = src[i];
+}
+
+cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int B, int rows,
+                           int H, int cap, int dst_row0, cudaStream_t stream) {
+  const long long row_vecs = static_cast<long long>(H) * HEAD_DIM * 2 / 16;
+  const long long span = row_vecs * rows;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // about 8 resident blocks of 256 threads per SM over the 2*B spans
+  long long want = (static_cast<long long>(sms) * 8 + 2 * B - 1) / (2 * B);
+  long long need = (span + 256 * 4 - 1) / (256 * 4);
+  int gx = static_cast<int>(want < need ? want : need);
+  if (gx < 1) gx = 1;
+  dim3 grid(gx, 2 * B);
+  kv_copy_kernel<<<grid, 256, 0, stream>>>(
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(ck),
+      static_cast<uint4*>(cv), B, span, span, row_vecs * cap, row_vecs * dst_row0);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Standalone 3D rotary embedding.  One block per token (b, s): its position is
+// computed once; the block's threads rotate the token's H*16 16-byte chunks.
+// ---------------------------------------------------------------------------
+// x and y may be the same buffer (in place): each thread reads and then writes
+// the same 16 bytes, so they are not declared __restrict__.
+__global__ void __launch_bounds__(128) rope3d_kernel(const uint4* x, uint4* y, int S, int H,
+                                                     ChunkGeom g, int first_chunk,
+                                                     RopeTables r) {
+  const long long token = blockIdx.x;  // b * S + s
+  const int s = static_cast<int>(token % S);
+  int t, hh, w;
+  token_pos(g, s, first_chunk, t, hh, w);
+  const int nvec = H * (HEAD_DIM / 8);
+  const uint4* src = x + token * nvec;
+  uint4* dst = y + token * nvec;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    const int j0 = (i & 15) * 4;
+    dst[i] = rope_chunk(src[i], r, j0, t, hh, w);
+  }
+}
+
+cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const ChunkGeom& g,
+                          int first_chunk, const RopeTables& r, cudaStream_t stream) {
+  const long long tokens = static_cast<long long>(B) * S;
+  if (tokens <= 0) return cudaSuccess;
+  rope3d_kernel<<<static_cast<unsigned>(tokens), 128, 0, stream>>>(
+      static_cast<const uint4*>(x), static_cast<uint4*>(y), S, H, g, first_chunk, r);
+  return cudaGetLastError();
+}
+
+}  // namespace dz

@@ -54,6 +54,7 @@ invariants, golden fixtures).  No function here is "parity unpinned".
 from __future__ import annotations
 
 import dataclasses
+import functools
 import math
 from typing import Optional, Tuple
 
@@ -110,11 +111,13 @@ def token_position(s: int, F: int, gh: int, gw: int, n_action: int, t_offset: in
     return t_offset + n * F, 0, 0
 
 
+@functools.lru_cache(maxsize=64)
 def token_positions(n_tokens: int, F: int, gh: int, gw: int, n_action: int,
                     t_offset: int, first_chunk: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """Arrays (t, h, w) of ``token_position`` for tokens 0..n_tokens-1."""
+    """Arrays (t, h, w) of ``token_position`` for tokens 0..n_tokens-1 (read-only)."""
     pos = np.array([token_position(s, F, gh, gw, n_action, t_offset, first_chunk)
                     for s in range(n_tokens)], dtype=np.int64).reshape(n_tokens, 3)
+    pos.setflags(write=False)
     return pos[:, 0], pos[:, 1], pos[:, 2]
 
 
@@ -224,6 +227,48 @@ def masked_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray,
     return out
 
 
+def rotated_operands(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
+                     mode: int, F: int, gh: int, gw: int, n_action: int, num_chunks: int,
+                     t_offset: int = 0, cache_k_bits: Optional[np.ndarray] = None,
+                     cache_v_bits: Optional[np.ndarray] = None, cache_len: int = 0,
+                     spec: RopeSpec = RopeSpec(), heads: Optional[slice] = None,
+                     batch: Optional[slice] = None):
+    """The call's q, keys and values as float64, rotated, keys in the call's order.
+
+    Rotary is applied to q and to the call's own k: DECODE at the positions of
+    chunk ``num_chunks``; PREFILL from chunk 0; TEACHER_FORCING with clean chunk
+    i and noisy chunk i both at chunk i's positions; never in CROSS.  Cache keys
+    are stored rotated and are used as they are, placed before the chunk's own
+    keys.  ``heads`` / ``batch`` optionally select a slice of heads / batch items.
+    """
+    L = chunk_len(F, gh, gw, n_action)
+    hs = slice(None) if heads is None else heads
+    bs = slice(None) if batch is None else batch
+    q = widen_bf16(q_bits[bs, :, hs, :])
+    k = widen_bf16(k_bits[bs, :, hs, :])
+    v = widen_bf16(v_bits[bs, :, hs, :])
+    if mode == DECODE:
+        q = rope3d(q, F, gh, gw, n_action, t_offset, num_chunks, spec)
+        k = rope3d(k, F, gh, gw, n_action, t_offset, num_chunks, spec)
+        if cache_len > 0:
+            ck = widen_bf16(cache_k_bits[bs, :cache_len, hs, :])
+            cv = widen_bf16(cache_v_bits[bs, :cache_len, hs, :])
+            k = np.concatenate([ck, k], axis=1)
+            v = np.concatenate([cv, v], axis=1)
+    elif mode == PREFILL:
+        q = rope3d(q, F, gh, gw, n_action, t_offset, 0, spec)
+        k = rope3d(k, F, gh, gw, n_action, t_offset, 0, spec)
+    elif mode == TEACHER_FORCING:
+        half = num_chunks * L
+        q = np.concatenate([rope3d(q[:, :half], F, gh, gw, n_action, t_offset, 0, spec),
+                            rope3d(q[:, half:], F, gh, gw, n_action, t_offset, 0, spec)], axis=1)
+        k = np.concatenate([rope3d(k[:, :half], F, gh, gw, n_action, t_offset, 0, spec),
+                            rope3d(k[:, half:], F, gh, gw, n_action, t_offset, 0, spec)], axis=1)
+    elif mode != CROSS:
+        raise ValueError(f"unknown mode {mode}")
+    return q, k, v
+
+
 def chunk_attn_forward(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
                        mode: int, F: int, gh: int, gw: int, n_action: int,
                        num_chunks: int, t_offset: int = 0, kv_len: int = 0,
@@ -233,38 +278,12 @@ def chunk_attn_forward(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarra
                        heads: Optional[slice] = None) -> np.ndarray:
     """dz_chunk_attn_forward on bf16 bit arrays; returns float64 [B, Sq, H, D].
 
-    Rotary is applied to q and to the call's own k (not to cache keys, which
-    are stored rotated; not in CROSS mode).  ``heads`` optionally restricts the
-    computation to a slice of heads (the result then holds only those heads).
+    ``heads`` optionally restricts the computation to a slice of heads (the
+    result then holds only those heads).
     """
     L = chunk_len(F, gh, gw, n_action)
-    sel = slice(None) if heads is None else heads
-    q = widen_bf16(q_bits)[:, :, sel, :]
-    k = widen_bf16(k_bits)[:, :, sel, :]
-    v = widen_bf16(v_bits)[:, :, sel, :]
-    if mode == DECODE:
-        q = rope3d(q, F, gh, gw, n_action, t_offset, num_chunks, spec)
-        k = rope3d(k, F, gh, gw, n_action, t_offset, num_chunks, spec)
-        if cache_len > 0:
-            ck = widen_bf16(cache_k_bits[:, :cache_len])[:, :, sel, :]
-            cv = widen_bf16(cache_v_bits[:, :cache_len])[:, :, sel, :]
-            k = np.concatenate([ck, k], axis=1)
-            v = np.concatenate([cv, v], axis=1)
-    elif mode == PREFILL:
-        q = rope3d(q, F, gh, gw, n_action, t_offset, 0, spec)
-        k = rope3d(k, F, gh, gw, n_action, t_offset, 0, spec)
-    elif mode == TEACHER_FORCING:
-        N = num_chunks
-        half = N * L
-        # clean chunks take positions 0..N-1, noisy chunk i takes clean chunk i's
-        q = np.concatenate([rope3d(q[:, :half], F, gh, gw, n_action, t_offset, 0, spec),
-                            rope3d(q[:, half:], F, gh, gw, n_action, t_offset, 0, spec)], axis=1)
-        k = np.concatenate([rope3d(k[:, :half], F, gh, gw, n_action, t_offset, 0, spec),
-                            rope3d(k[:, half:], F, gh, gw, n_action, t_offset, 0, spec)], axis=1)
-    elif mode == CROSS:
-        pass
-    else:
-        raise ValueError(f"unknown mode {mode}")
+    q, k, v = rotated_operands(q_bits, k_bits, v_bits, mode, F, gh, gw, n_action, num_chunks,
+                               t_offset, cache_k_bits, cache_v_bits, cache_len, spec, heads)
     vis = visibility(mode, L, num_chunks, cache_len=cache_len, kv_len=kv_len)
     assert vis.shape == (q.shape[1], k.shape[1]), (vis.shape, q.shape, k.shape)
     return masked_attention(q, k, v, vis)
@@ -282,42 +301,17 @@ def attention_rows(q_bits, k_bits, v_bits, rows, mode: int, F: int, gh: int, gw:
     L = chunk_len(F, gh, gw, n_action)
     D = q_bits.shape[-1]
     out = np.empty((len(rows), D), dtype=np.float64)
-    vis_cache = {}
+    vis = visibility(mode, L, num_chunks, cache_len=cache_len, kv_len=kv_len)
+    groups = {}
     for n, (b, s, h) in enumerate(rows):
-        qrow = widen_bf16(q_bits[b:b + 1, s:s + 1, h:h + 1, :])
-        kk = widen_bf16(k_bits[b:b + 1, :, h:h + 1, :])
-        vv = widen_bf16(v_bits[b:b + 1, :, h:h + 1, :])
-        if mode == DECODE:
-            qrow = rope3d_single(qrow, s, F, gh, gw, n_action, t_offset, num_chunks, spec)
-            kk = rope3d(kk, F, gh, gw, n_action, t_offset, num_chunks, spec)
-            if cache_len > 0:
-                ck = widen_bf16(cache_k_bits[b:b + 1, :cache_len, h:h + 1, :])
-                cv = widen_bf16(cache_v_bits[b:b + 1, :cache_len, h:h + 1, :])
-                kk = np.concatenate([ck, kk], axis=1)
-                vv = np.concatenate([cv, vv], axis=1)
-        elif mode == PREFILL:
-            qrow = rope3d_single(qrow, s, F, gh, gw, n_action, t_offset, 0, spec)
-            kk = rope3d(kk, F, gh, gw, n_action, t_offset, 0, spec)
-        elif mode == TEACHER_FORCING:
-            half = num_chunks * L
-            qrow = rope3d_single(qrow, s % half, F, gh, gw, n_action, t_offset, 0, spec)
-            kk = np.concatenate([rope3d(kk[:, :half], F, gh, gw, n_action, t_offset, 0, spec),
-                                 rope3d(kk[:, half:], F, gh, gw, n_action, t_offset, 0, spec)],
-                                axis=1)
-        key = (mode, L, num_chunks, cache_len, kv_len)
-        if key not in vis_cache:
-            vis_cache[key] = visibility(mode, L, num_chunks, cache_len=cache_len, kv_len=kv_len)
-        vis_row = vis_cache[key][s:s + 1]
-        out[n] = masked_attention(qrow, kk, vv, vis_row)[0, 0, 0]
+        groups.setdefault((b, h), []).append((n, s))
+    for (b, h), items in groups.items():
+        q, k, v = rotated_operands(q_bits, k_bits, v_bits, mode, F, gh, gw, n_action, num_chunks,
+                                   t_offset, cache_k_bits, cache_v_bits, cache_len, spec,
+                                   heads=slice(h, h + 1), batch=slice(b, b + 1))
+        for n, s in items:
+            out[n] = masked_attention(q[:, s:s + 1], k, v, vis[s:s + 1])[0, 0, 0]
     return out
-
-
-def rope3d_single(x: np.ndarray, s: int, F: int, gh: int, gw: int, n_action: int,
-                  t_offset: int, first_chunk: int, spec: RopeSpec) -> np.ndarray:
-    """Rotate a single token (x [1, 1, H, D]) that sits at index s of its run."""
-    t, h, w = token_position(s, F, gh, gw, n_action, t_offset, first_chunk)
-    theta = rope_angles(np.array([t]), np.array([h]), np.array([w]), spec)
-    return rotate_pairs(x, theta)
 
 
 # ---------------------------------------------------------------------------

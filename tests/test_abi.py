@@ -1,0 +1,90 @@
+"""Host-side tests of the C ABI (no GPU): the library loads, exports every entry
+point include/dz.h declares, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from causal_video_diffusion_rope_b200 import build, dz
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return dz.load()
+
+
+def _declared_functions():
+    names = set()
+    include = os.path.join(ROOT, "include")
+    for f in os.listdir(include):
+        if not f.endswith(".h"):
+            continue
+        text = open(os.path.join(include, f)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*(dz_[A-Za-z0-9_]+)\s*\(",
+                             text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared_functions()
+    assert {"dz_attn_create", "dz_chunk_attn_forward", "dz_rope3d", "dz_kvcache_append",
+            "dz_kvcache_replace"} <= declared
+    for name in declared:
+        assert hasattr(lib, name), f"libdz.so does not export {name}"
+    assert set(dz.EXPORTS) <= declared
+
+
+def test_status_strings(lib):
+    assert dz.status_string(0) == "ok"
+    for s in range(1, 8):
+        assert dz.status_string(s) not in ("ok", "unknown status")
+    assert dz.status_string(99) == "unknown status"
+
+
+def test_create_rejects_bad_descriptors(lib):
+    h = ctypes.c_void_p()
+    assert lib.dz_attn_create(ctypes.byref(h), None) == dz.DZ_ERR_INVALID_ARG
+    d = dz.make_desc()
+    d.head_dim = 64
+    assert lib.dz_attn_create(ctypes.byref(h), ctypes.byref(d)) == dz.DZ_ERR_SHAPE
+    d = dz.make_desc(pairs=(22, 21, 20))
+    assert lib.dz_attn_create(ctypes.byref(h), ctypes.byref(d)) == dz.DZ_ERR_SHAPE
+    d = dz.make_desc(num_heads=0)
+    assert lib.dz_attn_create(ctypes.byref(h), ctypes.byref(d)) == dz.DZ_ERR_SHAPE
+    d = dz.make_desc(max_q_tokens=2048 * 256 + 1)
+    assert lib.dz_attn_create(ctypes.byref(h), ctypes.byref(d)) == dz.DZ_ERR_CAPACITY
+    d = dz.make_desc(rope_base=1.0)
+    assert lib.dz_attn_create(ctypes.byref(h), ctypes.byref(d)) == dz.DZ_ERR_SHAPE
+
+
+def test_calls_reject_null_handle(lib):
+    lay = dz.make_layout(dz.DZ_MODE_DECODE, 1, 2, 11, 20, 24, 4)
+    cache = dz.make_cache(16, 16, 1, 10, 0, 464)
+    assert lib.dz_chunk_attn_forward(None, 16, 16, 16, None, ctypes.byref(lay), 16, None) == \
+        dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_rope3d(None, 16, 16, 1, 1, ctypes.byref(lay), 0, None) == dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_kvcache_append(None, ctypes.byref(cache), 16, 16, None) == dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_kvcache_replace(None, ctypes.byref(cache), 0, 16, 16, None) == \
+        dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_attn_sync_status(None, None) == dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_attn_destroy(None) == dz.DZ_ERR_INVALID_ARG
+
+
+def test_python_binding_raises(lib):
+    with pytest.raises(dz.DzError) as e:
+        d = dz.make_desc()
+        d.head_dim = 96
+        dz.dz_attn_create(d)
+    assert e.value.status == dz.DZ_ERR_SHAPE
+
+
+def test_binding_has_same_names_as_header():
+    declared = _declared_functions()
+    for name in declared:
+        assert hasattr(dz, name), f"binding lacks {name}"

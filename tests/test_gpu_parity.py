@@ -1,0 +1,371 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Attention: max |gpu - ref| <= 2e-2 and relative L2 <= 5e-3 per call.
+Rotary: per element |gpu - ref| <= 2^-8 |ref| + 2^-20 (|x0| + |x1|) (one bf16
+rounding of an fp32 rotation).  Cache append/replace: bit-exact.
+"""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+from causal_video_diffusion_rope_b200 import dz, synth
+from causal_video_diffusion_rope_b200.synth import (Layout, MODE_CROSS, MODE_DECODE, MODE_PREFILL,
+                                                    MODE_TEACHER_FORCING, WORKLOADS)
+from gpu_util import Handle, assert_close, to_bits, to_dev, to_f64
+from oracle import dz_oracle as O
+
+pytestmark = pytest.mark.gpu
+
+D = 128
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dz.load()
+
+
+_handles = {}
+
+
+def handle(heads):
+    if heads not in _handles:
+        _handles[heads] = Handle(heads)
+    return _handles[heads].h
+
+
+def teardown_module(module):
+    for h in _handles.values():
+        h.close()
+    _handles.clear()
+
+
+def rand_bits(rng, shape, scale=1.0):
+    return synth.bf16_bits_from_f32(rng.standard_normal(shape).astype(np.float32) * scale)
+
+
+def run_forward(lay: Layout, heads: int, q, k, v, cache_k=None, cache_v=None, cache_len=0):
+    h = handle(heads)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    cache = None
+    keep = []
+    if lay.mode == MODE_DECODE and cache_k is not None:
+        ck, cv = to_dev(cache_k), to_dev(cache_v)
+        keep += [ck, cv]
+        cache = dz.make_cache(ck, cv, lay.batch, cache_k.shape[1], cache_len, lay.chunk_len)
+    out = torch.empty((lay.batch, lay.q_len, heads, D), dtype=torch.bfloat16, device="cuda")
+    dz.dz_chunk_attn_forward(h, qd, kd, vd, cache, dz.layout_from(lay), out)
+    dz.dz_attn_sync_status(h)
+    return to_f64(out)
+
+
+def oracle_full(lay: Layout, q, k, v, cache_k=None, cache_v=None, cache_len=0):
+    return O.chunk_attn_forward(q, k, v, lay.mode, lay.frames_per_chunk, lay.grid_h, lay.grid_w,
+                                lay.n_action, lay.num_chunks, t_offset=lay.t_offset,
+                                kv_len=lay.kv_len, cache_k_bits=cache_k, cache_v_bits=cache_v,
+                                cache_len=cache_len)
+
+
+def oracle_rows(lay: Layout, rows, q, k, v, cache_k=None, cache_v=None, cache_len=0):
+    return O.attention_rows(q, k, v, rows, lay.mode, lay.frames_per_chunk, lay.grid_h,
+                            lay.grid_w, lay.n_action, lay.num_chunks, t_offset=lay.t_offset,
+                            kv_len=lay.kv_len, cache_k_bits=cache_k, cache_v_bits=cache_v,
+                            cache_len=cache_len)
+
+
+# ------------------------------------------------------------------ cache ops
+
+@pytest.mark.parametrize("B,H,L,chunks", [(1, 40, 464, 5), (2, 40, 464, 9), (2, 3, 36, 4),
+                                          (1, 1, 1, 7)])
+def test_kvcache_append_replace_bit_exact(B, H, L, chunks):
+    rng = np.random.default_rng(100 + L)
+    h = handle(H)
+    cap = chunks * L + 3
+    ck = torch.zeros((B, cap, H, D), dtype=torch.bfloat16, device="cuda")
+    cv = torch.zeros((B, cap, H, D), dtype=torch.bfloat16, device="cuda")
+    ref_k = np.zeros((B, cap, H, D), dtype=np.uint16)
+    ref_v = np.zeros((B, cap, H, D), dtype=np.uint16)
+    cache = dz.make_cache(ck, cv, B, cap, 0, L)
+    n = 0
+    for c in range(chunks):
+        k = rand_bits(rng, (B, L, H, D))
+        v = rand_bits(rng, (B, L, H, D))
+        dz.dz_kvcache_append(h, cache, to_dev(k), to_dev(v))
+        n = O.kvcache_append(ref_k, ref_v, n, k, v)
+        assert cache.len_tokens == n
+    torch.cuda.synchronize()
+    assert np.array_equal(to_bits(ck), ref_k) and np.array_equal(to_bits(cv), ref_v)
+    # replace the last chunk and one in the middle
+    for c in (chunks - 1, chunks // 2):
+        k = rand_bits(rng, (B, L, H, D))
+        v = rand_bits(rng, (B, L, H, D))
+        dz.dz_kvcache_replace(h, cache, c, to_dev(k), to_dev(v))
+        O.kvcache_replace(ref_k, ref_v, c, L, k, v)
+    torch.cuda.synchronize()
+    assert cache.len_tokens == n
+    assert np.array_equal(to_bits(ck), ref_k) and np.array_equal(to_bits(cv), ref_v)
+    # capacity: one more chunk does not fit -> error, nothing written
+    before = to_bits(ck)
+    k = rand_bits(rng, (B, L, H, D))
+    if n + L > cap:
+        with pytest.raises(dz.DzError) as e:
+            dz.dz_kvcache_append(h, cache, to_dev(k), to_dev(k))
+        assert e.value.status == dz.DZ_ERR_CAPACITY
+        assert cache.len_tokens == n
+        torch.cuda.synchronize()
+        assert np.array_equal(to_bits(ck), before)
+    with pytest.raises(dz.DzError) as e:
+        dz.dz_kvcache_replace(h, cache, chunks, to_dev(k), to_dev(k))
+    assert e.value.status == dz.DZ_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ rotary
+
+@pytest.mark.parametrize("B,S,H,F,gh,gw,na,t0,first", [
+    (1, 108, 2, 1, 4, 8, 4, 0, 0),
+    (1, 464, 40, 2, 11, 20, 24, 0, 4),
+    (2, 928, 3, 2, 11, 20, 24, 5, 31),
+    (1, 37, 1, 1, 1, 1, 0, 100, 0),
+])
+def test_rope3d_matches_oracle(B, S, H, F, gh, gw, na, t0, first):
+    rng = np.random.default_rng(7 + S)
+    x = rand_bits(rng, (B, S, H, D), 2.0)
+    h = handle(H)
+    lay = dz.make_layout(0, B, F, gh, gw, na, 0, t0)
+    xd = to_dev(x)
+    y = torch.empty_like(xd)
+    dz.dz_rope3d(h, xd, y, B, S, lay, first)
+    got = to_f64(y)
+    xf = O.widen_bf16(x)
+    ref = O.rope3d(xf, F, gh, gw, na, t0, first)
+    pair_mag = np.repeat(np.abs(xf[..., 0::2]) + np.abs(xf[..., 1::2]), 2, axis=-1)
+    bound = 2.0 ** -8 * np.abs(ref) + 2.0 ** -20 * pair_mag
+    assert (np.abs(got - ref) <= bound).all(), float(np.abs(got - ref).max())
+    # in place gives the same bytes
+    dz.dz_rope3d(h, xd, xd, B, S, lay, first)
+    torch.cuda.synchronize()
+    assert torch.equal(xd.view(torch.int16), y.view(torch.int16))
+
+
+def test_rope3d_rejects_positions_beyond_tables():
+    h = handle(2)
+    x = torch.zeros((1, 36, 2, D), dtype=torch.bfloat16, device="cuda")
+    lay = dz.make_layout(0, 1, 1, 4, 8, 4, 0, 4090)
+    with pytest.raises(dz.DzError) as e:
+        dz.dz_rope3d(h, x, x, 1, 72, lay, 10)
+    assert e.value.status == dz.DZ_ERR_SHAPE
+
+
+# ------------------------------------------------------------------ attention, element-wise
+
+def L_(mode, B, F, gh, gw, na, N, t0=0, kv=0):
+    return Layout(mode, B, F, gh, gw, na, N, t0, kv)
+
+
+SMALL_CASES = [
+    # name, layout, heads, cache_len, q/k scale
+    ("tiny_prefill_c0", WORKLOADS[0].layout, 2, 0, 1.0),
+    ("decode_L464_cache1856_h4", L_(MODE_DECODE, 1, 2, 11, 20, 24, 4), 4, 1856, 1.0),
+    ("decode_no_cache", L_(MODE_DECODE, 1, 2, 11, 20, 24, 0), 3, 0, 1.0),
+    ("decode_L36_cache300_b2", L_(MODE_DECODE, 2, 1, 4, 8, 4, 9, 3), 3, 300, 1.0),
+    ("decode_cache_one_tile_b2", L_(MODE_DECODE, 2, 1, 4, 8, 4, 3), 2, 128, 1.0),
+    ("decode_L464_cache3712_scaled", L_(MODE_DECODE, 1, 2, 11, 20, 24, 8), 2, 3712, 3.0),
+    ("tf_N2_L464", L_(MODE_TEACHER_FORCING, 1, 2, 11, 20, 24, 2), 2, 0, 1.0),
+    ("tf_N3_L36", L_(MODE_TEACHER_FORCING, 1, 1, 4, 8, 4, 3), 2, 0, 1.0),
+    ("tf_N4_L100_b2", L_(MODE_TEACHER_FORCING, 2, 1, 9, 10, 10, 4, 2), 2, 0, 1.0),
+    ("prefill_N5_L100", L_(MODE_PREFILL, 1, 1, 9, 10, 10, 5), 2, 0, 1.0),
+    ("prefill_L1_N130", L_(MODE_PREFILL, 1, 1, 1, 1, 0, 130), 1, 0, 1.0),
+    ("prefill_N3_L256_scaled", L_(MODE_PREFILL, 1, 1, 16, 16, 0, 3), 2, 0, 4.0),
+    ("cross_464x769_b2", L_(MODE_CROSS, 2, 2, 11, 20, 24, 1, 0, 769), 2, 0, 1.0),
+    ("cross_kv1", L_(MODE_CROSS, 1, 1, 4, 8, 4, 2, 0, 1), 2, 0, 1.0),
+    ("cross_kv5000", L_(MODE_CROSS, 1, 1, 4, 8, 4, 1, 0, 5000), 2, 0, 1.0),
+]
+
+
+@pytest.mark.parametrize("name,lay,heads,cache_len,scale", SMALL_CASES,
+                         ids=[c[0] for c in SMALL_CASES])
+def test_attention_elementwise(name, lay, heads, cache_len, scale):
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    B = lay.batch
+    q = rand_bits(rng, (B, lay.q_len, heads, D), scale)
+    k = rand_bits(rng, (B, lay.self_kv_len, heads, D), scale)
+    v = rand_bits(rng, (B, lay.self_kv_len, heads, D))
+    ck = cv = None
+    if lay.mode == MODE_DECODE and cache_len > 0:
+        cap = cache_len + 77
+        ck = np.full((B, cap, heads, D), 0x7FC1, dtype=np.uint16)  # NaN past the cached rows
+        cv = np.full((B, cap, heads, D), 0x7FC1, dtype=np.uint16)
+        ck[:, :cache_len] = rand_bits(rng, (B, cache_len, heads, D), scale)
+        cv[:, :cache_len] = rand_bits(rng, (B, cache_len, heads, D))
+    got = run_forward(lay, heads, q, k, v, ck, cv, cache_len)
+    ref = oracle_full(lay, q, k, v, ck, cv, cache_len)
+    assert_close(got, ref, name)
+
+
+def test_single_visible_key_exact():
+    """Chunks of one token: query 0 sees only key 0, so out[0] is v[0] exactly."""
+    rng = np.random.default_rng(3)
+    lay = L_(MODE_PREFILL, 1, 1, 1, 1, 0, 200)
+    q = rand_bits(rng, (1, 200, 2, D))
+    k = rand_bits(rng, (1, 200, 2, D))
+    v = rand_bits(rng, (1, 200, 2, D))
+    got = run_forward(lay, 2, q, k, v)
+    assert np.array_equal(got[:, 0], O.widen_bf16(v)[:, 0])
+
+
+def test_repeatable_bitwise():
+    w = WORKLOADS[1]
+    inp = synth.make_inputs(w, 11)
+    a = run_forward(w.layout, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
+                    inp["cache_v"], w.cache_tokens)
+    b = run_forward(w.layout, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
+                    inp["cache_v"], w.cache_tokens)
+    assert np.array_equal(a, b)
+
+
+def test_decode_matches_prefill_last_chunk():
+    """DECODE over a cache of rotated (dz_rope3d) chunks == PREFILL's last-chunk rows."""
+    rng = np.random.default_rng(21)
+    F, gh, gw, na, n, H = 1, 8, 8, 8, 3, 2
+    lay_p = L_(MODE_PREFILL, 1, F, gh, gw, na, n + 1)
+    L = lay_p.chunk_len
+    q = rand_bits(rng, (1, (n + 1) * L, H, D))
+    k = rand_bits(rng, (1, (n + 1) * L, H, D))
+    v = rand_bits(rng, (1, (n + 1) * L, H, D))
+    full = run_forward(lay_p, H, q, k, v)
+    h = handle(H)
+    kd = to_dev(k[:, :n * L])
+    krot = torch.empty_like(kd)
+    dz.dz_rope3d(h, kd, krot, 1, n * L, dz.make_layout(0, 1, F, gh, gw, na, 0), 0)
+    lay_d = L_(MODE_DECODE, 1, F, gh, gw, na, n)
+    dec = run_forward(lay_d, H, q[:, n * L:], k[:, n * L:], v[:, n * L:], to_bits(krot),
+                      v[:, :n * L], n * L)
+    assert_close(dec, full[:, n * L:], "decode vs prefill")
+
+
+def test_forward_argument_errors():
+    h = handle(2)
+    lay = dz.make_layout(MODE_DECODE, 1, 1, 4, 8, 4, 0)
+    x = torch.zeros((1, 64, 2, D), dtype=torch.bfloat16, device="cuda")
+    bad = x.data_ptr() + 2
+    with pytest.raises(dz.DzError) as e:
+        dz.dz_chunk_attn_forward(h, bad, x, x, None, lay, x)
+    assert e.value.status == dz.DZ_ERR_ALIGNMENT
+    lay_far = dz.make_layout(MODE_DECODE, 1, 1, 4, 8, 4, 5000)
+    with pytest.raises(dz.DzError) as e:
+        dz.dz_chunk_attn_forward(h, x, x, x, None, lay_far, x)
+    assert e.value.status == dz.DZ_ERR_SHAPE
+    lay_b = dz.make_layout(MODE_DECODE, 3, 1, 4, 8, 4, 0)
+    with pytest.raises(dz.DzError) as e:
+        dz.dz_chunk_attn_forward(h, x, x, x, None, lay_b, x)
+    assert e.value.status == dz.DZ_ERR_CAPACITY
+
+
+# ------------------------------------------------------------------ the five workloads at full size
+
+def sample_rows(rng, B, Sq, H, boosted, L, n_random=48):
+    specials = [0, 1, 127, 128, 255, 256, 383, 384, L - 1, Sq - 1]
+    specials += [c * L + d for c in range(1, Sq // L) for d in (-1, 0)]
+    rows = set()
+    for s in specials:
+        if 0 <= s < Sq:
+            rows.add((int(rng.integers(B)), s, int(rng.integers(H))))
+    for hh in boosted:
+        rows.add((int(rng.integers(B)), int(rng.integers(Sq)), int(hh)))
+    for _ in range(n_random):
+        rows.add((int(rng.integers(B)), int(rng.integers(Sq)), int(rng.integers(H))))
+    return sorted(rows)
+
+
+def check_rows(got, ref_rows, rows, what):
+    g = np.array([got[b, s, h] for b, s, h in rows])
+    assert_close(g, ref_rows, what)
+
+
+def test_workload0_tiny_prefill():
+    w = WORKLOADS[0]
+    inp = synth.make_inputs(w, 0)
+    got = run_forward(w.layout, w.heads, inp["q"], inp["k"], inp["v"])
+    assert_close(got, oracle_full(w.layout, inp["q"], inp["k"], inp["v"]), w.name)
+
+
+def test_workload1_decode_full_elementwise():
+    w = WORKLOADS[1]
+    inp = synth.make_inputs(w, 1)
+    got = run_forward(w.layout, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
+                      inp["cache_v"], w.cache_tokens)
+    ref = oracle_full(w.layout, inp["q"], inp["k"], inp["v"], inp["cache_k"], inp["cache_v"],
+                      w.cache_tokens)
+    assert_close(got, ref, w.name)
+
+
+def test_workload2_cfg_denoise_loop_with_replace():
+    """16 denoising steps per request with fresh q/k/v, the last cached chunk replaced
+    by an observed chunk between requests; 3 requests."""
+    w = WORKLOADS[2]
+    lay = w.layout
+    B, H, L = lay.batch, w.heads, lay.chunk_len
+    inp = synth.make_inputs(w, 2)
+    ck_host, cv_host = inp["cache_k"].copy(), inp["cache_v"].copy()
+    h = handle(H)
+    ck, cv = to_dev(ck_host), to_dev(cv_host)
+    cache = dz.make_cache(ck, cv, B, ck_host.shape[1], w.cache_tokens, L)
+    rng = np.random.default_rng(1234)
+    out = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda")
+    for req in range(3):
+        for step in range(w.denoise_steps):
+            x = synth.fresh_chunk(rng, w)
+            dz.dz_chunk_attn_forward(h, to_dev(x["q"]), to_dev(x["k"]), to_dev(x["v"]), cache,
+                                     dz.layout_from(lay), out)
+            dz.dz_attn_sync_status(h)
+            got = to_f64(out)
+            if step in (0, w.denoise_steps - 1) and req != 1:
+                ref = oracle_full(lay, x["q"], x["k"], x["v"], ck_host, cv_host, w.cache_tokens)
+                assert_close(got, ref, f"request {req} step {step}")
+            else:
+                rows = sample_rows(rng, B, L, H, [], L, n_random=12)
+                ref = oracle_rows(lay, rows, x["q"], x["k"], x["v"], ck_host, cv_host,
+                                  w.cache_tokens)
+                check_rows(got, ref, rows, f"request {req} step {step}")
+        # the real observation replaces the last chunk
+        obs_k = synth.normal_bf16(rng, (B, L, H, D))
+        obs_v = synth.normal_bf16(rng, (B, L, H, D))
+        last = w.cache_tokens // L - 1
+        dz.dz_kvcache_replace(h, cache, last, to_dev(obs_k), to_dev(obs_v))
+        O.kvcache_replace(ck_host, cv_host, last, L, obs_k, obs_v)
+        torch.cuda.synchronize()
+        assert np.array_equal(to_bits(ck), ck_host) and np.array_equal(to_bits(cv), cv_host)
+
+
+def test_workload3_teacher_forcing_sampled():
+    w = WORKLOADS[3]
+    lay = w.layout
+    inp = synth.make_inputs(w, 3)
+    got = run_forward(lay, w.heads, inp["q"], inp["k"], inp["v"])
+    rng = np.random.default_rng(33)
+    rows = sample_rows(rng, 1, lay.q_len, w.heads, [], lay.chunk_len, n_random=96)
+    ref = oracle_rows(lay, rows, inp["q"], inp["k"], inp["v"])
+    check_rows(got, ref, rows, w.name)
+    assert np.isfinite(got).all()
+
+
+def test_workload4_long_cache_and_cross():
+    w = WORKLOADS[4]
+    lay = w.layout
+    inp = synth.make_inputs(w, 4)
+    got = run_forward(lay, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
+                      inp["cache_v"], w.cache_tokens)
+    rng = np.random.default_rng(44)
+    rows = sample_rows(rng, lay.batch, lay.q_len, w.heads, inp["boosted_heads"],
+                       lay.chunk_len, n_random=64)
+    ref = oracle_rows(lay, rows, inp["q"], inp["k"], inp["v"], inp["cache_k"], inp["cache_v"],
+                      w.cache_tokens)
+    check_rows(got, ref, rows, w.name + " self")
+    assert np.isfinite(got).all()
+    xl = synth.cross_layout(w)
+    gx = run_forward(xl, w.heads, inp["q_x"], inp["k_x"], inp["v_x"])
+    rx = oracle_full(xl, inp["q_x"], inp["k_x"], inp["v_x"])
+    assert_close(gx, rx, w.name + " cross")
