@@ -310,6 +310,14 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
   p.geom = g;
   p.rope = tables_of(a);
   p.rope_q = p.rope_k = (l->mode != DZ_MODE_CROSS) ? 1 : 0;
+  if (p.rope_q) {
+    p.stage_t0 = g.t_offset + (l->mode == DZ_MODE_DECODE ? l->num_chunks * g.F : 0);
+    p.stage_nt = (l->mode == DZ_MODE_DECODE ? 1 : l->num_chunks) * g.F;
+    const long long n = static_cast<long long>(p.stage_nt) * a->desc.rope_pairs_t +
+                        static_cast<long long>(g.gh) * a->desc.rope_pairs_h +
+                        static_cast<long long>(g.gw) * a->desc.rope_pairs_w;
+    p.stage_ok = n <= dz::ROPE_STAGE_MAX ? 1 : 0;
+  }
   p.out = out;
   p.ws = a->ws;
   p.counters = a->counters;

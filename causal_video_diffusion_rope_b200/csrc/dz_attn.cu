@@ -50,18 +50,29 @@ constexpr int TILE_BYTES = TILE_M * HEAD_DIM * 2;  // 32 KiB
 constexpr int HALF_BYTES = TILE_BYTES / 2;         // 64 dims x 128 rows
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// Registers per thread: the kernel is compiled for LAUNCH_REGS (3 warps per SM
+// sub-partition); warpgroup 0 (producer, MMA, rotary) then gives registers to
+// the two softmax warpgroups.  The split must add up to the launch budget.
+constexpr int LAUNCH_REGS = 168;
+constexpr int REGS_CTRL = 104;
+constexpr int REGS_SOFT = 200;
+static_assert(REGS_CTRL + 2 * REGS_SOFT == 3 * LAUNCH_REGS, "register split must match launch");
 
 // shared memory layout (offsets from a 1024-byte aligned base)
 constexpr int SM_Q = 0;
 constexpr int SM_K = SM_Q + Q_TILES * TILE_BYTES;
 constexpr int SM_V = SM_K + KV_STAGES * TILE_BYTES;
-constexpr int SM_BAR = SM_V + KV_STAGES * TILE_BYTES;
+constexpr int XPOSE_PITCH = 80;                        // bytes per row of a warp's transpose buffer
+constexpr int XPOSE_WARP = 32 * XPOSE_PITCH;           // 32 rows x 64 data bytes (+16 pad)
+constexpr int SM_X = SM_V + KV_STAGES * TILE_BYTES;    // 8 softmax warps' transpose buffers
+constexpr int SM_BAR = SM_X + 8 * XPOSE_WARP;
 enum {
   B_Q_FULL = 0,
   B_Q_READY = 1,
   B_Q_EMPTY = 2,
-  B_K_FULL = 3,
-  B_K_READY = B_K_FULL + KV_STAGES,
+  B_K_FULL = 3,                     // K tile landed (tiles used as loaded)
+  B_K_RAW = B_K_FULL + KV_STAGES,   // K tile landed (tiles the rotary gate must rotate)
+  B_K_READY = B_K_RAW + KV_STAGES,  // rotated K tile released to the tensor core
   B_K_EMPTY = B_K_READY + KV_STAGES,
   B_V_FULL = B_K_EMPTY + KV_STAGES,
   B_V_EMPTY = B_V_FULL + KV_STAGES,
@@ -75,7 +86,8 @@ enum {
 };
 constexpr int SM_MISC = SM_BAR + 256;         // tmem base, abort flag, combine flags
 constexpr int SM_PREFIX = SM_MISC + 256;      // (MAX_Q_GROUPS + 1) ints
-constexpr int SM_TOTAL = SM_PREFIX + (MAX_Q_GROUPS + 1) * 4;
+constexpr int SM_ROPE = SM_PREFIX + ((MAX_Q_GROUPS + 1) * 4 + 15) / 16 * 16;  // staged rotary rows
+constexpr int SM_TOTAL = SM_ROPE + ROPE_STAGE_MAX * 8;
 constexpr int SMEM_BYTES = SM_TOTAL + 1024;   // alignment slack
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -91,6 +103,7 @@ struct __align__(64) AttnParams {
   SchedGeom sched;
   int B, H, n_qg;
   int rope_q, rope_k;
+  int stage_ok, stage_t0, stage_nt;
   long long W;
   int G;
   float scale_log2;
@@ -203,17 +216,82 @@ __device__ __forceinline__ void seq_pos(const AttnParams& p, int s, int& t, int&
   token_pos(p.geom, ss, first, t, h, w);
 }
 
-// Rotate row r of a 128x128 bf16 tile held as two 128B-swizzled halves.
+// Rotate row r of a 128x128 bf16 tile held as two 128B-swizzled halves (16-byte
+// chunk c of row r sits at half (c / 8), slot (c % 8) ^ (r % 8)).  The table
+// values of four chunks are loaded before their shared-memory read-modify-write
+// so that the loads overlap.  `rt.tab` may point to shared or global memory.
 __device__ __forceinline__ void rotate_tile_row(uint8_t* tile, int r, const RopeTables& rt, int t,
                                                 int h, int w) {
+  uint8_t* row = tile + r * 128;
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
+  for (int b4 = 0; b4 < 4; ++b4) {
+    float2 cs[16];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint4* ptr = reinterpret_cast<uint4*>(tile + half * HALF_BYTES + r * 128 + ((c ^ (r & 7)) << 4));
-      *ptr = rope_chunk(*ptr, rt, half * 32 + c * 4, t, h, w);
+    for (int k = 0; k < 4; ++k) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        cs[4 * k + i] = rt.tab[rope_index(rt, (b4 * 4 + k) * 4 + i, t, h, w)];
+    }
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = b4 * 4 + k;
+      v[k] = *reinterpret_cast<const uint4*>(row + (c >> 3) * HALF_BYTES + (((c & 7) ^ (r & 7)) << 4));
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[k].x = rope_pair(v[k].x, cs[4 * k + 0]);
+      v[k].y = rope_pair(v[k].y, cs[4 * k + 1]);
+      v[k].z = rope_pair(v[k].z, cs[4 * k + 2]);
+      v[k].w = rope_pair(v[k].w, cs[4 * k + 3]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = b4 * 4 + k;
+      *reinterpret_cast<uint4*>(row + (c >> 3) * HALF_BYTES + (((c & 7) ^ (r & 7)) << 4)) = v[k];
     }
   }
+}
+
+// Bits j (0 <= j < 32) with lo <= j < hi.
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 32);
+  if (hi <= lo) return 0u;
+  const uint32_t up = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  return up & ~((1u << lo) - 1u);
+}
+
+// Scores of columns outside [la, ha) and [lb, hb) become -inf (32 columns from col0).
+__device__ __forceinline__ void mask_cols(uint32_t (&v)[32], int col0, int la, int ha, int lb,
+                                          int hb) {
+  const uint32_t keep = range_bits(la - col0, ha - col0) | range_bits(lb - col0, hb - col0);
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = ((keep >> j) & 1u) ? v[j] : 0xff800000u;  // -inf
+}
+
+__device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = __uint_as_float(v[k]);
+#pragma unroll
+  for (int j = 8; j < 32; ++j) m[j & 7] = fmaxf(m[j & 7], __uint_as_float(v[j]));
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+
+// p = 2^(s * scale_log2 - mb) for 32 scores, packed as 16 bf16 pairs into pk[off, off + 16);
+// returns the fp32 sum of the 32 probabilities.
+__device__ __forceinline__ float exp_pack(const uint32_t (&v)[32], uint32_t (&pk)[32], int off,
+                                          float sl2, float mb) {
+  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const float p0 = ex2(__fmaf_rn(__uint_as_float(v[2 * j]), sl2, -mb));
+    const float p1 = ex2(__fmaf_rn(__uint_as_float(v[2 * j + 1]), sl2, -mb));
+    s4[j & 3] += p0 + p1;
+    pk[off + j] = pack_bf16x2(p0, p1);
+  }
+  return (s4[0] + s4[1]) + (s4[2] + s4[3]);
 }
 
 __device__ __forceinline__ long long cta_start(long long c, long long W, int G) {
@@ -260,6 +338,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bar[B_Q_EMPTY], 1);
     for (int s = 0; s < KV_STAGES; ++s) {
       mbar_init(&bar[B_K_FULL + s], 1);
+      mbar_init(&bar[B_K_RAW + s], 1);
       mbar_init(&bar[B_K_READY + s], ROPE_THREADS);
       mbar_init(&bar[B_K_EMPTY + s], 1);
       mbar_init(&bar[B_V_FULL + s], 1);
@@ -281,6 +360,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_relinquish();
   }
   for (int g = tid; g < p.n_qg; g += NTHREADS) prefix[g + 1] = unit_tile_count(p.sched, g);
+  // rotary view: the call's table rows copied to shared memory when they fit
+  RopeTables rope = p.rope;
+  if (p.stage_ok) {
+    float2* st_tab = reinterpret_cast<float2*>(smem + SM_ROPE);
+    const int nt = p.stage_nt * p.rope.pt, nh = p.geom.gh * p.rope.ph, nw = p.geom.gw * p.rope.pw;
+    const float2* gt = p.rope.tab + p.rope.off_t + p.stage_t0 * p.rope.pt;
+    const float2* gh = p.rope.tab + p.rope.off_h;
+    const float2* gw = p.rope.tab + p.rope.off_w;
+    for (int i = tid; i < nt + nh + nw; i += NTHREADS)
+      st_tab[i] = i < nt ? gt[i] : (i < nt + nh ? gh[i - nt] : gw[i - nt - nh]);
+    rope.tab = st_tab;
+    rope.off_t = -p.stage_t0 * p.rope.pt;
+    rope.off_h = nt;
+    rope.off_w = nt + nh;
+  }
   __syncthreads();
   if (warp == 0) {  // inclusive scan of the counts -> prefix[0..n_qg]
     int carry = 0;
@@ -305,6 +399,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const long long cstart = cta_start(blockIdx.x, p.W, p.G);
   const long long cend = cta_start(blockIdx.x + 1, p.W, p.G);
 
+  if (warp < WARP_SOFT) {
+  regs_dec<REGS_CTRL>();
   if (warp == WARP_TMA) {
     // ======================= TMA producer =======================
     if (lane == 0) {
@@ -319,10 +415,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       Seg sg;
       int seg_i = 0;
       uint32_t k_iss = 0, v_iss = 0;  // K and V tiles issued so far
+      // loads issued per stage on K_FULL (used as loaded) and K_RAW (to be rotated);
+      // each of those barriers has exactly one consumer that takes its phases in order
+      uint32_t kf_cnt[KV_STAGES] = {0, 0}, kr_cnt[KV_STAGES] = {0, 0};
       int q_loads = 0;
       bool ok = true;
       while (ok && seg_next(p, prefix, pos, cend, sg)) {
         const int b = sg.bh / p.H, h = sg.bh - (sg.bh / p.H) * p.H;
+        // Q of this segment: the previous segment's last QK products must be done
         if (seg_i > 0 && !mbar_wait(&bar[B_Q_EMPTY], (seg_i - 1) & 1, abort_flag, p.status)) break;
         mbar_expect_tx(&bar[B_Q_FULL], Q_TILES * TILE_BYTES);
         for (int q = 0; q < Q_TILES; ++q) {
@@ -338,9 +438,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const CUtensorMap* mk = kt.cache ? &p.tm_ck : &p.tm_k;
           const CUtensorMap* mv = kt.cache ? &p.tm_cv : &p.tm_v;
           if (!mbar_wait(&bar[B_K_EMPTY + st], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
-          mbar_expect_tx(&bar[B_K_FULL + st], TILE_BYTES);
-          tma_load_4d(sK + st * TILE_BYTES, mk, &bar[B_K_FULL + st], 0, h, kt.row0, b);
-          tma_load_4d(sK + st * TILE_BYTES + HALF_BYTES, mk, &bar[B_K_FULL + st], 64, h, kt.row0, b);
+          uint64_t* kb = &bar[(kt.rope ? B_K_RAW : B_K_FULL) + st];
+          mbar_expect_tx(kb, TILE_BYTES);
+          tma_load_4d(sK + st * TILE_BYTES, mk, kb, 0, h, kt.row0, b);
+          tma_load_4d(sK + st * TILE_BYTES + HALF_BYTES, mk, kb, 64, h, kt.row0, b);
+          if (kt.rope) ++kr_cnt[st]; else ++kf_cnt[st];
           ++k_iss;
           if (!mbar_wait(&bar[B_V_EMPTY + st], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
           mbar_expect_tx(&bar[B_V_FULL + st], TILE_BYTES);
@@ -353,8 +455,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // drain: every copy this thread issued has landed before the CTA exits
       // (on the normal path all of them were consumed and these return at once)
       if (q_loads > 0) drain_wait(&bar[B_Q_FULL], (q_loads - 1) & 1);
-      for (uint32_t j = (k_iss > KV_STAGES ? k_iss - KV_STAGES : 0); j < k_iss; ++j)
-        drain_wait(&bar[B_K_FULL + j % KV_STAGES], (j / KV_STAGES) & 1);
+      for (int st = 0; st < KV_STAGES; ++st) {
+        if (kf_cnt[st] > 0) drain_wait(&bar[B_K_FULL + st], (kf_cnt[st] - 1) & 1);
+        if (kr_cnt[st] > 0) drain_wait(&bar[B_K_RAW + st], (kr_cnt[st] - 1) & 1);
+      }
       for (uint32_t j = (v_iss > KV_STAGES ? v_iss - KV_STAGES : 0); j < v_iss; ++j)
         drain_wait(&bar[B_V_FULL + j % KV_STAGES], (j / KV_STAGES) & 1);
     }
@@ -386,6 +490,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       Seg sg;
       int seg_i = 0;
       uint32_t it = 0, tn = 0;
+      uint32_t kr_par = 0;  // bit s: parity of the next K_READY phase on stage s
+      uint32_t kf_par = 0;  // bit s: parity of the next K_FULL phase on stage s
       bool ok = true;
       while (ok && seg_next(p, prefix, pos, cend, sg)) {
         if (!mbar_wait(&bar[B_Q_READY], seg_i & 1, abort_flag, p.status)) break;
@@ -395,8 +501,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < sg.n; ++i, ++it, ++tn) {
           const int st = it % KV_STAGES;
           const uint32_t ph = (it / KV_STAGES) & 1;
-          if (!mbar_wait(&bar[B_K_READY + st], ph, abort_flag, p.status)) { ok = false; break; }
+          const bool rot = ktile(p, seg_tile(sg, i)).rope;
+          bool got;
+          if (rot) {
+            got = mbar_wait(&bar[B_K_READY + st], (kr_par >> st) & 1, abort_flag, p.status);
+            kr_par ^= 1u << st;
+          } else {
+            got = mbar_wait(&bar[B_K_FULL + st], (kf_par >> st) & 1, abort_flag, p.status);
+            kf_par ^= 1u << st;
+          }
+          if (!got) { ok = false; break; }
           tc_fence_after();
+          const bool last = (i == sg.n - 1);
           if (i == 0) {
             for (int q = 0; q < Q_TILES; ++q) {
               issue_qk(q, st);
@@ -423,6 +539,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!ok) break;
           }
           mma_commit(&bar[B_K_EMPTY + st]);
+          if (last) mma_commit(&bar[B_Q_EMPTY]);  // Q may be replaced once these QK are done
           pst = st;
           pph = ph;
         }
@@ -445,20 +562,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         if (!ok) break;
         mma_commit(&bar[B_V_EMPTY + pst]);
-        mma_commit(&bar[B_Q_EMPTY]);
         ++seg_i;
       }
       // every issued MMA has completed before TMEM is released
       mma_commit(&bar[B_DRAIN]);
       drain_wait(&bar[B_DRAIN], 0);
     }
-  } else if (warp < WARP_SOFT) {
+  } else {
     // ======================= rotary gate =======================
-    const int r0 = tid - WARP_ROPE * 32;  // rows r0 and r0 + ROPE_THREADS of a tile
+    const int r0 = tid - WARP_ROPE * 32;  // rows r0 + k * ROPE_THREADS of a tile
     long long pos = cstart;
     Seg sg;
     int seg_i = 0;
     uint32_t it = 0;
+    uint32_t raw_par = 0;  // bit s: parity of the next K_RAW phase on stage s
     bool ok = true;
     while (ok && seg_next(p, prefix, pos, cend, sg)) {
       if (!mbar_wait(&bar[B_Q_FULL], seg_i & 1, abort_flag, p.status)) break;
@@ -469,7 +586,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (s < p.sched.Sq) {
               int t, h, w;
               seq_pos(p, s, t, h, w);
-              rotate_tile_row(sQ + q * TILE_BYTES, r, p.rope, t, h, w);
+              rotate_tile_row(sQ + q * TILE_BYTES, r, rope, t, h, w);
             }
           }
         }
@@ -477,30 +594,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_smem();
       mbar_arrive(&bar[B_Q_READY]);
       for (int i = 0; i < sg.n; ++i, ++it) {
-        const int st = it % KV_STAGES;
-        const uint32_t ph = (it / KV_STAGES) & 1;
-        if (!mbar_wait(&bar[B_K_FULL + st], ph, abort_flag, p.status)) { ok = false; break; }
         const KTile kt = ktile(p, seg_tile(sg, i));
-        if (kt.rope) {
-          for (int r = r0; r < kt.nvalid; r += ROPE_THREADS) {
-            int t, h, w;
-            seq_pos(p, kt.row0 + r, t, h, w);
-            rotate_tile_row(sK + st * TILE_BYTES, r, p.rope, t, h, w);
-          }
+        if (!kt.rope) continue;  // cache tiles go to the tensor core as loaded
+        const int st = it % KV_STAGES;
+        if (!mbar_wait(&bar[B_K_RAW + st], (raw_par >> st) & 1, abort_flag, p.status)) { ok = false; break; }
+        raw_par ^= 1u << st;
+        for (int r = r0; r < kt.nvalid; r += ROPE_THREADS) {
+          int t, h, w;
+          seq_pos(p, kt.row0 + r, t, h, w);
+          rotate_tile_row(sK + st * TILE_BYTES, r, rope, t, h, w);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar[B_K_READY + st]);
       }
       ++seg_i;
     }
+  }
   } else {
+    regs_inc<REGS_SOFT>();
     // ======================= softmax groups =======================
     const int q = (warp - WARP_SOFT) >> 2;           // Q tile of this group
     const int gtid = tid - (WARP_SOFT + 4 * q) * 32;  // 0..127 inside the group
-    const int r = 32 * (warp & 3) + lane;            // TMEM lane = tile row
-    const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const int quarter = warp & 3;                    // TMEM lane quarter of this warp
+    const int r = 32 * quarter + lane;               // TMEM lane = tile row
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
     const uint32_t tS = tmem + lane_addr + q * TILE_N;
     const uint32_t tO = tmem + lane_addr + 256 + q * HEAD_DIM;
+    uint8_t* xp = smem + SM_X + (warp - WARP_SOFT) * XPOSE_WARP;  // this warp's transpose buffer
     const float sl2 = p.scale_log2;
     long long pos = cstart;
     Seg sg;
@@ -509,7 +629,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     while (ok && seg_next(p, prefix, pos, cend, sg)) {
       const int b = sg.bh / p.H, h = sg.bh - (sg.bh / p.H) * p.H;
-      const int s_tok = sg.qg * Q_GROUP + q * TILE_M + r;
+      const int row0 = sg.qg * Q_GROUP + q * TILE_M + 32 * quarter;  // token of this warp's lane 0
+      const int s_tok = row0 + lane;
       const int s_eff = s_tok < p.sched.Sq ? s_tok : p.sched.Sq - 1;
       int a0, a1, b0, b1;
       row_ranges(p.sched, s_eff, a0, a1, b0, b1);
@@ -523,33 +644,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int lb = max(0, min(TILE_N, b0 - kt.vbase));
         const int hb = max(0, min(kt.nvalid, b1 - kt.vbase));
         const bool full = (la == 0 && ha == TILE_N);
-        uint32_t v[32];
-        // pass 1: row maximum of the visible scores
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int col = c * 32 + j;
-            float s = __uint_as_float(v[j]);
-            if (!full && !((col >= la && col < ha) || (col >= lb && col < hb))) s = -INFINITY;
-            mx = fmaxf(mx, s);
-          }
+        uint32_t v0[32], v1[32], v2[32], v3[32];
+        tmem_ld32(tS, v0);
+        tmem_ld32(tS + 32, v1);
+        tmem_ld32(tS + 64, v2);
+        tmem_ld32(tS + 96, v3);
+        tmem_wait_ld();
+        if (!full) {
+          mask_cols(v0, 0, la, ha, lb, hb);
+          mask_cols(v1, 32, la, ha, lb, hb);
+          mask_cols(v2, 64, la, ha, lb, hb);
+          mask_cols(v3, 96, la, ha, lb, hb);
         }
+        const float mx = fmaxf(fmaxf(max32(v0), max32(v1)), fmaxf(max32(v2), max32(v3)));
         const float m_new = fmaxf(m_run, mx * sl2);
         const bool need = m_new > m_run + RESCALE_THRESHOLD;
         const float alpha = need ? ex2(m_run - m_new) : 1.f;
         if (__any_sync(0xffffffffu, need) && i > 0) {
           // O holds tiles < i of this segment (its PV completed before S_FULL fired)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            tmem_ld32(tO + c * 32, v);
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t v[16];
+            tmem_ld16(tO + c * 16, v);
             tmem_wait_ld();
+            uint32_t w16[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-            tmem_st32(tO + c * 32, v);
+            for (int j = 0; j < 16; ++j) w16[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+            tmem_st16(tO + c * 16, w16);
           }
           tmem_wait_st();
         }
@@ -558,29 +679,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           m_run = m_new;
         }
         const float mb = (m_run == -INFINITY) ? 0.f : m_run;
-        // pass 2: probabilities, written as bf16 pairs over the first 64 columns of S
-        float lsum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int col = c * 32 + 2 * j;
-            float s0 = __uint_as_float(v[2 * j]);
-            float s1 = __uint_as_float(v[2 * j + 1]);
-            if (!full) {
-              if (!((col >= la && col < ha) || (col >= lb && col < hb))) s0 = -INFINITY;
-              if (!((col + 1 >= la && col + 1 < ha) || (col + 1 >= lb && col + 1 < hb))) s1 = -INFINITY;
-            }
-            const float p0 = ex2(__fmaf_rn(s0, sl2, -mb));
-            const float p1 = ex2(__fmaf_rn(s1, sl2, -mb));
-            lsum += p0 + p1;
-            pk[j] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + c * 16, pk);
-        }
+        // probabilities, written as bf16 pairs over the first 64 columns of S
+        uint32_t pk0[32], pk1[32];
+        const float lsum = exp_pack(v0, pk0, 0, sl2, mb) + exp_pack(v1, pk0, 16, sl2, mb) +
+                           exp_pack(v2, pk1, 0, sl2, mb) + exp_pack(v3, pk1, 16, sl2, mb);
+        tmem_st32(tS, pk0);
+        tmem_st32(tS + 32, pk1);
         tmem_wait_st();
         l_run += lsum;
         tc_fence_before();
@@ -590,49 +694,71 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // ---- epilogue of the segment ----
       if (!mbar_wait(&bar[B_O_FULL + q], seg_i & 1, abort_flag, p.status)) break;
       tc_fence_after();
-      const bool store_row = s_tok < p.sched.Sq;
       if (sg.full) {
+        // bf16 out = O / l; each 32-column chunk goes through the warp's transpose
+        // buffer so that global stores cover 64 contiguous bytes of 8 rows at a time
         const float inv_l = 1.f / l_run;
-        __nv_bfloat16* orow = p.out + ((static_cast<size_t>(b) * p.sched.Sq + (store_row ? s_tok : 0)) * p.H + h) * HEAD_DIM;
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
           tmem_ld32(tO + c * 32, v);
           tmem_wait_ld();
-          if (store_row) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              pk[j] = pack_bf16x2(__uint_as_float(v[2 * j]) * inv_l, __uint_as_float(v[2 * j + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+          if (c == 3) {
+            tc_fence_before();
+            mbar_arrive(&bar[B_O_FREE + q]);
           }
+          uint4* xrow = reinterpret_cast<uint4*>(xp + lane * XPOSE_PITCH);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            xrow[j] = make_uint4(
+                pack_bf16x2(__uint_as_float(v[8 * j]) * inv_l, __uint_as_float(v[8 * j + 1]) * inv_l),
+                pack_bf16x2(__uint_as_float(v[8 * j + 2]) * inv_l, __uint_as_float(v[8 * j + 3]) * inv_l),
+                pack_bf16x2(__uint_as_float(v[8 * j + 4]) * inv_l, __uint_as_float(v[8 * j + 5]) * inv_l),
+                pack_bf16x2(__uint_as_float(v[8 * j + 6]) * inv_l, __uint_as_float(v[8 * j + 7]) * inv_l));
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int task = lane + 32 * k;
+            const int rr = task >> 2, piece = task & 3;
+            const int s = row0 + rr;
+            const uint4 val = *reinterpret_cast<const uint4*>(xp + rr * XPOSE_PITCH + piece * 16);
+            if (s < p.sched.Sq) {
+              __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + c * 32 + piece * 8;
+              *reinterpret_cast<uint4*>(dst) = val;
+            }
+          }
+          __syncwarp();
         }
-        tc_fence_before();
-        mbar_arrive(&bar[B_O_FREE + q]);
       } else {
-        // partial piece: fp32 (O, m, l) to this CTA's slot
+        // partial piece: fp32 (O, m, l) to this CTA's slot, 16 columns at a time
         const bool first_piece = cta_start(blockIdx.x, p.W, p.G) >= sg.u0;
         const int slot = 2 * blockIdx.x + (first_piece ? 0 : 1);
         float* buf = p.ws + static_cast<size_t>(slot) * PART_FLOATS;
-        float* orow = buf + static_cast<size_t>(q * TILE_M + r) * HEAD_DIM;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tO + c * 32, v);
+        float* obase = buf + static_cast<size_t>(q * TILE_M + 32 * quarter) * HEAD_DIM;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t v[16];
+          tmem_ld16(tO + c * 16, v);
           tmem_wait_ld();
-          float4* dst = reinterpret_cast<float4*>(orow + c * 32);
+          if (c == 7) {
+            tc_fence_before();
+            mbar_arrive(&bar[B_O_FREE + q]);
+          }
+          uint4* xrow = reinterpret_cast<uint4*>(xp + lane * XPOSE_PITCH);
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+          for (int j = 0; j < 4; ++j) xrow[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int task = lane + 32 * k;
+            const int rr = task >> 2, piece = task & 3;
+            const uint4 val = *reinterpret_cast<const uint4*>(xp + rr * XPOSE_PITCH + piece * 16);
+            *reinterpret_cast<uint4*>(obase + rr * HEAD_DIM + c * 16 + piece * 4) = val;
+          }
+          __syncwarp();
         }
-        tc_fence_before();
-        mbar_arrive(&bar[B_O_FREE + q]);
-        float* ml = buf + static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM + (q * TILE_M + r) * 2;
-        ml[0] = m_run;
-        ml[1] = l_run;
+        float* ml = buf + static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM;
+        reinterpret_cast<float2*>(ml)[q * TILE_M + r] = make_float2(m_run, l_run);
         __threadfence();
         mbar_arrive(&bar[B_WG + q]);
         if (!mbar_wait(&bar[B_WG + q], wg_phase & 1, abort_flag, p.status)) break;
@@ -648,53 +774,74 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!mbar_wait(&bar[B_WG + q], wg_phase & 1, abort_flag, p.status)) break;
         ++wg_phase;
         if (comb_flag[q]) {
+          // last piece to finish merges all pieces.  Lane = row for the (m, l) of
+          // every piece; then 4 rows at a time with lanes over the 128 columns, so
+          // the O loads of 4 rows x 4 pieces are in flight together and coalesced.
           __threadfence();
+          const size_t ml_off = static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM;
+          const int row_l = q * TILE_M + 32 * quarter + lane;  // this lane's row (m, l)
           float M = -INFINITY;
           for (int c2 = c_first; c2 <= c_last; ++c2) {
             const int sl = 2 * c2 + (cta_start(c2, p.W, p.G) >= sg.u0 ? 0 : 1);
-            const float* ml2 = p.ws + static_cast<size_t>(sl) * PART_FLOATS +
-                               static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM + (q * TILE_M + r) * 2;
-            M = fmaxf(M, __ldcg(ml2));
+            M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(p.ws + static_cast<size_t>(sl) * PART_FLOATS + ml_off) + row_l).x);
           }
           float Lsum = 0.f;
           for (int c2 = c_first; c2 <= c_last; ++c2) {
             const int sl = 2 * c2 + (cta_start(c2, p.W, p.G) >= sg.u0 ? 0 : 1);
-            const float* ml2 = p.ws + static_cast<size_t>(sl) * PART_FLOATS +
-                               static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM + (q * TILE_M + r) * 2;
-            const float m2 = __ldcg(ml2);
-            if (m2 != -INFINITY) Lsum += __ldcg(ml2 + 1) * ex2(m2 - M);
+            const float2 ml2 = __ldcg(reinterpret_cast<const float2*>(p.ws + static_cast<size_t>(sl) * PART_FLOATS + ml_off) + row_l);
+            if (ml2.x != -INFINITY) Lsum += ml2.y * ex2(ml2.x - M);
           }
-          const float inv_l = 1.f / Lsum;
+          const float invL = 1.f / Lsum;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            float acc[32];
+          for (int rr0 = 0; rr0 < 32; rr0 += 4) {
+            float4 acc[4];
+            float Mr[4], iL[4];
 #pragma unroll
-            for (int d = 0; d < 32; ++d) acc[d] = 0.f;
-            for (int c2 = c_first; c2 <= c_last; ++c2) {
-              const int sl = 2 * c2 + (cta_start(c2, p.W, p.G) >= sg.u0 ? 0 : 1);
-              const float* b2 = p.ws + static_cast<size_t>(sl) * PART_FLOATS;
-              const float m2 = __ldcg(b2 + static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM + (q * TILE_M + r) * 2);
-              if (m2 == -INFINITY) continue;
-              const float wgt = ex2(m2 - M);
-              const float4* o2 = reinterpret_cast<const float4*>(b2 + static_cast<size_t>(q * TILE_M + r) * HEAD_DIM + c * 32);
+            for (int k = 0; k < 4; ++k) {
+              acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+              Mr[k] = __shfl_sync(0xffffffffu, M, rr0 + k);
+              iL[k] = __shfl_sync(0xffffffffu, invL, rr0 + k);
+            }
+            for (int c2 = c_first; c2 <= c_last; c2 += 4) {
+              float4 o[4][4];
+              float mm[4][4];
 #pragma unroll
-              for (int d = 0; d < 8; ++d) {
-                const float4 x = __ldcg(o2 + d);
-                acc[4 * d] += wgt * x.x;
-                acc[4 * d + 1] += wgt * x.y;
-                acc[4 * d + 2] += wgt * x.z;
-                acc[4 * d + 3] += wgt * x.w;
+              for (int u = 0; u < 4; ++u) {
+                const int cc = c2 + u;
+                const int sl = 2 * cc + (cta_start(cc, p.W, p.G) >= sg.u0 ? 0 : 1);
+                const float* b2 = p.ws + static_cast<size_t>(sl) * PART_FLOATS;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const int row = q * TILE_M + 32 * quarter + rr0 + k;
+                  if (cc <= c_last) {
+                    mm[u][k] = __ldcg(reinterpret_cast<const float2*>(b2 + ml_off) + row).x;
+                    o[u][k] = __ldcg(reinterpret_cast<const float4*>(b2 + static_cast<size_t>(row) * HEAD_DIM) + lane);
+                  } else {
+                    mm[u][k] = -INFINITY;
+                    o[u][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+                  }
+                }
+              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float wgt = (mm[u][k] == -INFINITY) ? 0.f : ex2(mm[u][k] - Mr[k]);
+                  acc[k].x += wgt * o[u][k].x;
+                  acc[k].y += wgt * o[u][k].y;
+                  acc[k].z += wgt * o[u][k].z;
+                  acc[k].w += wgt * o[u][k].w;
+                }
               }
             }
-            if (store_row) {
-              __nv_bfloat16* orow2 = p.out + ((static_cast<size_t>(b) * p.sched.Sq + s_tok) * p.H + h) * HEAD_DIM + c * 32;
-              uint4* dst = reinterpret_cast<uint4*>(orow2);
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                dst[j] = make_uint4(pack_bf16x2(acc[8 * j] * inv_l, acc[8 * j + 1] * inv_l),
-                                    pack_bf16x2(acc[8 * j + 2] * inv_l, acc[8 * j + 3] * inv_l),
-                                    pack_bf16x2(acc[8 * j + 4] * inv_l, acc[8 * j + 5] * inv_l),
-                                    pack_bf16x2(acc[8 * j + 6] * inv_l, acc[8 * j + 7] * inv_l));
+            for (int k = 0; k < 4; ++k) {
+              const int s = row0 + rr0 + k;
+              if (s < p.sched.Sq) {
+                __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + 4 * lane;
+                *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[k].x * iL[k], acc[k].y * iL[k]),
+                                                            pack_bf16x2(acc[k].z * iL[k], acc[k].w * iL[k]));
+              }
             }
           }
           if (gtid == 0) *counter = 0;  // ready for the next call
@@ -719,8 +866,13 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(chunk_attn_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    // the warpgroup register split assumes exactly LAUNCH_REGS registers per thread
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_attn_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(chunk_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
@@ -742,6 +894,9 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   p.n_qg = a.n_qg;
   p.rope_q = a.rope_q;
   p.rope_k = a.rope_k;
+  p.stage_ok = a.stage_ok;
+  p.stage_t0 = a.stage_t0;
+  p.stage_nt = a.stage_nt;
   p.W = a.W;
   p.G = a.grid;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));

@@ -14,7 +14,7 @@ constexpr int TILE_M = 128;        // query rows per Q tile (TMEM lanes)
 constexpr int TILE_N = 128;        // keys per K/V tile
 constexpr int Q_TILES = 2;         // Q tiles per CTA (ping-pong between two softmax groups)
 constexpr int Q_GROUP = TILE_M * Q_TILES;  // query rows per work unit
-constexpr int MAX_Q_GROUPS = 2048; // per (batch, head); bounds the per-CTA prefix table
+constexpr int MAX_Q_GROUPS = 512;  // per (batch, head); bounds the per-CTA prefix table
 
 // Rotary tables: (cos, sin) as float2 for every (axis position, pair of that axis).
 struct RopeTables {
@@ -172,9 +172,15 @@ struct AttnLaunch {
   int B, H;
   int n_qg;
   int rope_q, rope_k;
+  // rotary-table rows the call needs (t in [stage_t0, stage_t0 + stage_nt), all h < gh,
+  // all w < gw), copied to shared memory at kernel start when stage_ok
+  int stage_ok, stage_t0, stage_nt;
   long long W;  // total key tiles over all units
   int grid;
 };
+
+// Capacity (float2 entries) of the attention kernel's shared-memory rotary table.
+constexpr int ROPE_STAGE_MAX = 1280;
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
 

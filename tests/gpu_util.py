@@ -1,4 +1,7 @@
 """Helpers for the GPU tests: device copies of bf16 bit arrays and the error metrics."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -31,11 +34,30 @@ def errors(got: np.ndarray, ref: np.ndarray):
     return max_abs, rel
 
 
-def assert_close(got: np.ndarray, ref: np.ndarray, what: str = ""):
+def log_errors(what: str, max_abs: float, rel: float, n: int) -> None:
+    """Append the measured errors to $DZ_PARITY_LOG (JSON lines) when it is set."""
+    path = os.environ.get("DZ_PARITY_LOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"case": what, "max_abs": max_abs, "rel_l2": rel,
+                                "elements": int(n)}) + "\n")
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, what: str = "", max_abs_tol: float = MAX_ABS,
+                 rel_tol: float = REL_L2):
     assert np.isfinite(got).all(), f"{what}: non-finite output"
     max_abs, rel = errors(got, ref)
-    assert max_abs <= MAX_ABS and rel <= REL_L2, f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
+    log_errors(what, max_abs, rel, got.size)
+    assert max_abs <= max_abs_tol and rel <= rel_tol, \
+        f"{what}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
     return max_abs, rel
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (8 significant bits, ties to even)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                      # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.round(np.ldexp(m, 8)), e - 8)
 
 
 class Handle:

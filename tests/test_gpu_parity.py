@@ -13,7 +13,7 @@ import torch
 from causal_video_diffusion_rope_b200 import dz, synth
 from causal_video_diffusion_rope_b200.synth import (Layout, MODE_CROSS, MODE_DECODE, MODE_PREFILL,
                                                     MODE_TEACHER_FORCING, WORKLOADS)
-from gpu_util import Handle, assert_close, to_bits, to_dev, to_f64
+from gpu_util import Handle, assert_close, bf16_round, to_bits, to_dev, to_f64
 from oracle import dz_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -172,13 +172,11 @@ SMALL_CASES = [
     ("decode_no_cache", L_(MODE_DECODE, 1, 2, 11, 20, 24, 0), 3, 0, 1.0),
     ("decode_L36_cache300_b2", L_(MODE_DECODE, 2, 1, 4, 8, 4, 9, 3), 3, 300, 1.0),
     ("decode_cache_one_tile_b2", L_(MODE_DECODE, 2, 1, 4, 8, 4, 3), 2, 128, 1.0),
-    ("decode_L464_cache3712_scaled", L_(MODE_DECODE, 1, 2, 11, 20, 24, 8), 2, 3712, 3.0),
     ("tf_N2_L464", L_(MODE_TEACHER_FORCING, 1, 2, 11, 20, 24, 2), 2, 0, 1.0),
     ("tf_N3_L36", L_(MODE_TEACHER_FORCING, 1, 1, 4, 8, 4, 3), 2, 0, 1.0),
     ("tf_N4_L100_b2", L_(MODE_TEACHER_FORCING, 2, 1, 9, 10, 10, 4, 2), 2, 0, 1.0),
     ("prefill_N5_L100", L_(MODE_PREFILL, 1, 1, 9, 10, 10, 5), 2, 0, 1.0),
     ("prefill_L1_N130", L_(MODE_PREFILL, 1, 1, 1, 1, 0, 130), 1, 0, 1.0),
-    ("prefill_N3_L256_scaled", L_(MODE_PREFILL, 1, 1, 16, 16, 0, 3), 2, 0, 4.0),
     ("cross_464x769_b2", L_(MODE_CROSS, 2, 2, 11, 20, 24, 1, 0, 769), 2, 0, 1.0),
     ("cross_kv1", L_(MODE_CROSS, 1, 1, 4, 8, 4, 2, 0, 1), 2, 0, 1.0),
     ("cross_kv5000", L_(MODE_CROSS, 1, 1, 4, 8, 4, 1, 0, 5000), 2, 0, 1.0),
@@ -205,6 +203,42 @@ def test_attention_elementwise(name, lay, heads, cache_len, scale):
     assert_close(got, ref, name)
 
 
+SCALED_CASES = [
+    ("decode_L464_cache3712_x3", L_(MODE_DECODE, 1, 2, 11, 20, 24, 8), 2, 3712, 3.0),
+    ("prefill_N3_L256_x4", L_(MODE_PREFILL, 1, 1, 16, 16, 0, 3), 2, 0, 4.0),
+    ("tf_N2_L464_x3", L_(MODE_TEACHER_FORCING, 1, 2, 11, 20, 24, 2), 2, 0, 3.0),
+]
+
+
+@pytest.mark.parametrize("name,lay,heads,cache_len,scale", SCALED_CASES,
+                         ids=[c[0] for c in SCALED_CASES])
+def test_attention_wide_scores(name, lay, heads, cache_len, scale):
+    """q and k drawn with std `scale` (score std scale^2, up to 16): beyond the workloads'
+    distribution.  The kernel's declared operand precision is bf16 for the rotated q and k,
+    so the output is checked (1) with the standard tolerance against the definition applied
+    to the rotated q/k rounded to bf16, and (2) against the exact oracle within the bound
+    that rounding implies: relative L2 <= 5e-3 * scale^2 / 4 (max abs <= 2e-2 * scale^2)."""
+    rng = np.random.default_rng(zlib.crc32(name.encode()))
+    B = lay.batch
+    q = rand_bits(rng, (B, lay.q_len, heads, D), scale)
+    k = rand_bits(rng, (B, lay.self_kv_len, heads, D), scale)
+    v = rand_bits(rng, (B, lay.self_kv_len, heads, D))
+    ck = cv = None
+    if cache_len:
+        ck = rand_bits(rng, (B, cache_len, heads, D), scale)
+        cv = rand_bits(rng, (B, cache_len, heads, D))
+    got = run_forward(lay, heads, q, k, v, ck, cv, cache_len)
+    qr, kr, vr = O.rotated_operands(q, k, v, lay.mode, lay.frames_per_chunk, lay.grid_h,
+                                    lay.grid_w, lay.n_action, lay.num_chunks, lay.t_offset,
+                                    ck, cv, cache_len)
+    vis = O.visibility(lay.mode, lay.chunk_len, lay.num_chunks, cache_len=cache_len)
+    ref_rounded = O.masked_attention(bf16_round(qr), bf16_round(kr), vr, vis)
+    assert_close(got, ref_rounded, name + " vs bf16-operand reference")
+    ref = oracle_full(lay, q, k, v, ck, cv, cache_len)
+    assert_close(got, ref, name + " vs exact oracle", max_abs_tol=2e-2 * scale ** 2,
+                 rel_tol=5e-3 * scale ** 2 / 4)
+
+
 def test_single_visible_key_exact():
     """Chunks of one token: query 0 sees only key 0, so out[0] is v[0] exactly."""
     rng = np.random.default_rng(3)
@@ -216,14 +250,15 @@ def test_single_visible_key_exact():
     assert np.array_equal(got[:, 0], O.widen_bf16(v)[:, 0])
 
 
-def test_repeatable_bitwise():
-    w = WORKLOADS[1]
+@pytest.mark.parametrize("wi", [1, 0])
+def test_repeatable_bitwise(wi):
+    """Identical calls give identical bytes (the split combine sums pieces in a fixed order)."""
+    w = WORKLOADS[wi]
     inp = synth.make_inputs(w, 11)
-    a = run_forward(w.layout, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
-                    inp["cache_v"], w.cache_tokens)
-    b = run_forward(w.layout, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
-                    inp["cache_v"], w.cache_tokens)
-    assert np.array_equal(a, b)
+    args = (inp["q"], inp["k"], inp["v"], inp.get("cache_k"), inp.get("cache_v"), w.cache_tokens)
+    first = run_forward(w.layout, w.heads, *args)
+    for _ in range(4):
+        assert np.array_equal(run_forward(w.layout, w.heads, *args), first)
 
 
 def test_decode_matches_prefill_last_chunk():
@@ -340,16 +375,12 @@ def test_workload2_cfg_denoise_loop_with_replace():
         assert np.array_equal(to_bits(ck), ck_host) and np.array_equal(to_bits(cv), cv_host)
 
 
-def test_workload3_teacher_forcing_sampled():
+def test_workload3_teacher_forcing_full_elementwise():
     w = WORKLOADS[3]
     lay = w.layout
     inp = synth.make_inputs(w, 3)
     got = run_forward(lay, w.heads, inp["q"], inp["k"], inp["v"])
-    rng = np.random.default_rng(33)
-    rows = sample_rows(rng, 1, lay.q_len, w.heads, [], lay.chunk_len, n_random=96)
-    ref = oracle_rows(lay, rows, inp["q"], inp["k"], inp["v"])
-    check_rows(got, ref, rows, w.name)
-    assert np.isfinite(got).all()
+    assert_close(got, oracle_full(lay, inp["q"], inp["k"], inp["v"]), w.name)
 
 
 def test_workload4_long_cache_and_cross():
@@ -358,13 +389,12 @@ def test_workload4_long_cache_and_cross():
     inp = synth.make_inputs(w, 4)
     got = run_forward(lay, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
                       inp["cache_v"], w.cache_tokens)
-    rng = np.random.default_rng(44)
-    rows = sample_rows(rng, lay.batch, lay.q_len, w.heads, inp["boosted_heads"],
-                       lay.chunk_len, n_random=64)
-    ref = oracle_rows(lay, rows, inp["q"], inp["k"], inp["v"], inp["cache_k"], inp["cache_v"],
+    ref = oracle_full(lay, inp["q"], inp["k"], inp["v"], inp["cache_k"], inp["cache_v"],
                       w.cache_tokens)
-    check_rows(got, ref, rows, w.name + " self")
-    assert np.isfinite(got).all()
+    assert_close(got, ref, w.name + " self")
+    # the heads whose keys are scaled by 3 on their own (within the same bound)
+    hx = inp["boosted_heads"]
+    assert_close(got[:, :, hx], ref[:, :, hx], w.name + " self, K x3 heads")
     xl = synth.cross_layout(w)
     gx = run_forward(xl, w.heads, inp["q_x"], inp["k_x"], inp["v_x"])
     rx = oracle_full(xl, inp["q_x"], inp["k_x"], inp["v_x"])
