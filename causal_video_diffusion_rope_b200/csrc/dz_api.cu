@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -389,3 +390,156 @@ dz_status dz_attn_sync_status(dz_attn_t a, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Attention without any allocation, for callers that cannot call cudaMalloc.
+//
+// The scratch memory the attention kernel needs (fp32 partial results of split
+// work units, the split counters and a status word) lives in one file-scope
+// static device array, and the rotary tables in a second one; both are created
+// with the module, so every GPU that loads this library holds them until the
+// process exits.  On host code the array names are host-side stand-ins, not
+// device addresses: their device addresses are looked up once per device with
+// cudaGetSymbolAddress, with that device current.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int NOALLOC_SLOTS = 126;                 // partial-result slots (2 per CTA)
+constexpr size_t NOALLOC_WS_BYTES = NOALLOC_SLOTS * dz::PART_FLOATS * sizeof(float);
+constexpr size_t NOALLOC_COUNTERS = 65536;         // split counters
+constexpr size_t NOALLOC_SCRATCH_BYTES = NOALLOC_WS_BYTES + NOALLOC_COUNTERS * sizeof(int) + 256;
+constexpr size_t NOALLOC_ROPE_ENTRIES = 294912;    // (cos, sin) pairs of the rotary tables
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+static __device__ __align__(256) float2 g_noalloc_rope[NOALLOC_ROPE_ENTRIES];
+
+struct NoallocDevice {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch
+  float2* rope = nullptr;            // device address of g_noalloc_rope
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  bool tables = false;               // rotary tables hold `rot` below
+  double base = 0.0;
+  int pt = 0, ph = 0, pw = 0, mt = 0, mh = 0, mw = 0;
+};
+NoallocDevice g_noalloc[64];
+std::mutex g_noalloc_mu;
+
+}  // namespace
+
+extern "C" dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* d, const void* q,
+                                                   const void* k, const void* v,
+                                                   const dz_kvcache* cache,
+                                                   const dz_chunk_layout* layout, void* out,
+                                                   void* stream) {
+  if (!d || !layout) return DZ_ERR_INVALID_ARG;
+  if (d->head_dim != dz::HEAD_DIM || d->num_heads < 1 || d->num_heads > 256) return DZ_ERR_SHAPE;
+  if (d->rope_pairs_t < 0 || d->rope_pairs_h < 0 || d->rope_pairs_w < 0 ||
+      d->rope_pairs_t + d->rope_pairs_h + d->rope_pairs_w != dz::HEAD_DIM / 2)
+    return DZ_ERR_SHAPE;
+  if (!(d->rope_base > 1.0) || !std::isfinite(d->rope_base)) return DZ_ERR_SHAPE;
+  if (d->max_batch < 1 || d->max_q_tokens < 1 || d->max_pos_t < 1 || d->max_pos_h < 1 ||
+      d->max_pos_w < 1)
+    return DZ_ERR_SHAPE;
+  // sizes beyond what the static arrays hold are rejected
+  const long long n_qg_max = cdiv(d->max_q_tokens, dz::Q_GROUP);
+  if (n_qg_max > dz::MAX_Q_GROUPS ||
+      static_cast<long long>(d->max_batch) * d->num_heads * n_qg_max * dz::Q_TILES >
+          static_cast<long long>(NOALLOC_COUNTERS)) {
+    if (debug_on())
+      std::fprintf(stderr, "[dz] noalloc: batch x heads x query groups exceeds %zu counters\n",
+                   NOALLOC_COUNTERS);
+    return DZ_ERR_CAPACITY;
+  }
+  const long long n_tab = static_cast<long long>(d->max_pos_t) * d->rope_pairs_t +
+                          static_cast<long long>(d->max_pos_h) * d->rope_pairs_h +
+                          static_cast<long long>(d->max_pos_w) * d->rope_pairs_w;
+  if (n_tab > static_cast<long long>(NOALLOC_ROPE_ENTRIES)) {
+    if (debug_on())
+      std::fprintf(stderr, "[dz] noalloc: rotary tables need %lld entries, %zu available\n",
+                   n_tab, NOALLOC_ROPE_ENTRIES);
+    return DZ_ERR_CAPACITY;
+  }
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DZ_ERR_CUDA;
+  NoallocDevice& nd = g_noalloc[dev];
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!nd.ready) {
+      // once per device, with that device current: device addresses of the arrays
+      void* sp = nullptr;
+      void* rp = nullptr;
+      if (cudaGetSymbolAddress(&sp, g_noalloc_scratch) != cudaSuccess ||
+          cudaGetSymbolAddress(&rp, g_noalloc_rope) != cudaSuccess)
+        return DZ_ERR_CUDA;
+      cudaDriverEntryPointQueryResult qr;
+      void* fn = nullptr;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qr) !=
+              cudaSuccess ||
+          qr != cudaDriverEntryPointSuccess || !fn)
+        return DZ_ERR_CUDA;
+      if (cudaDeviceGetAttribute(&nd.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DZ_ERR_CUDA;
+      nd.scratch = static_cast<unsigned char*>(sp);
+      nd.rope = static_cast<float2*>(rp);
+      nd.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+      nd.ready = true;
+    }
+    if (!nd.tables || nd.base != d->rope_base || nd.pt != d->rope_pairs_t ||
+        nd.ph != d->rope_pairs_h || nd.pw != d->rope_pairs_w || nd.mt != d->max_pos_t ||
+        nd.mh != d->max_pos_h || nd.mw != d->max_pos_w) {
+      // (re)build the rotary tables for this rotary configuration: a synchronous copy
+      std::vector<float2> tab(static_cast<size_t>(n_tab));
+      size_t off = 0;
+      const int npos[3] = {d->max_pos_t, d->max_pos_h, d->max_pos_w};
+      const int npairs[3] = {d->rope_pairs_t, d->rope_pairs_h, d->rope_pairs_w};
+      for (int ax = 0; ax < 3; ++ax) {
+        for (int j = 0; j < npairs[ax]; ++j) {
+          const double omega = std::pow(d->rope_base, -2.0 * j / (2.0 * npairs[ax]));
+          for (int pp = 0; pp < npos[ax]; ++pp) {
+            const double th = static_cast<double>(pp) * omega;
+            tab[off + static_cast<size_t>(pp) * npairs[ax] + j] =
+                make_float2(static_cast<float>(std::cos(th)), static_cast<float>(std::sin(th)));
+          }
+        }
+        off += static_cast<size_t>(npos[ax]) * npairs[ax];
+      }
+      if (!tab.empty() && cudaMemcpy(nd.rope, tab.data(), tab.size() * sizeof(float2),
+                                     cudaMemcpyHostToDevice) != cudaSuccess)
+        return DZ_ERR_CUDA;
+      nd.tables = true;
+      nd.base = d->rope_base;
+      nd.pt = d->rope_pairs_t;
+      nd.ph = d->rope_pairs_h;
+      nd.pw = d->rope_pairs_w;
+      nd.mt = d->max_pos_t;
+      nd.mh = d->max_pos_h;
+      nd.mw = d->max_pos_w;
+    }
+  }
+
+  // a handle-shaped view of the static memory; the grid is capped so that each
+  // CTA's two partial-result slots fit in the static workspace
+  dz_attn a;
+  a.device = dev;
+  a.num_sms = nd.num_sms < NOALLOC_SLOTS / 2 ? nd.num_sms : NOALLOC_SLOTS / 2;
+  a.desc = *d;
+  a.rope_tab = nd.rope;
+  a.off_t = 0;
+  a.off_h = d->max_pos_t * d->rope_pairs_t;
+  a.off_w = a.off_h + d->max_pos_h * d->rope_pairs_h;
+  a.ws = reinterpret_cast<float*>(nd.scratch);
+  a.counters = reinterpret_cast<int*>(nd.scratch + NOALLOC_WS_BYTES);
+  a.n_counters = static_cast<size_t>(d->max_batch) * d->num_heads * n_qg_max * dz::Q_TILES;
+  a.status = reinterpret_cast<int*>(nd.scratch + NOALLOC_WS_BYTES + NOALLOC_COUNTERS * sizeof(int));
+  a.encode = nd.encode;
+  // the split counters and the status word must start at zero (a previous call that
+  // gave up may have left them set); cleared on the caller's stream
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(a.counters, 0, a.n_counters * sizeof(int), st) != cudaSuccess ||
+      cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess)
+    return DZ_ERR_CUDA;
+  return dz_chunk_attn_forward(&a, q, k, v, cache, layout, out, stream);
+}

@@ -33,6 +33,7 @@ DZ_MODE_CROSS = 3
 EXPORTS = [
     "dz_attn_create", "dz_attn_destroy", "dz_rope3d", "dz_chunk_attn_forward",
     "dz_kvcache_append", "dz_kvcache_replace", "dz_attn_sync_status", "dz_status_string",
+    "dz_chunk_attn_forward_noalloc",
 ]
 
 
@@ -90,6 +91,9 @@ def load() -> ctypes.CDLL:
     lib.dz_rope3d.argtypes = [vp, vp, vp, i32, i32, ctypes.POINTER(dz_chunk_layout), i32, vp]
     lib.dz_chunk_attn_forward.argtypes = [vp, vp, vp, vp, ctypes.POINTER(dz_kvcache),
                                           ctypes.POINTER(dz_chunk_layout), vp, vp]
+    lib.dz_chunk_attn_forward_noalloc.argtypes = [
+        ctypes.POINTER(dz_attn_desc), vp, vp, vp, ctypes.POINTER(dz_kvcache),
+        ctypes.POINTER(dz_chunk_layout), vp, vp]
     lib.dz_kvcache_append.argtypes = [vp, ctypes.POINTER(dz_kvcache), vp, vp, vp]
     lib.dz_kvcache_replace.argtypes = [vp, ctypes.POINTER(dz_kvcache), i32, vp, vp, vp]
     lib.dz_attn_sync_status.argtypes = [vp, vp]
@@ -177,6 +181,16 @@ def dz_chunk_attn_forward(handle: int, q, k, v, cache: Optional[dz_kvcache],
     _check(load().dz_chunk_attn_forward(handle, _ptr(q), _ptr(k), _ptr(v), cptr,
                                         ctypes.byref(layout), _ptr(out), _stream(stream)),
            "dz_chunk_attn_forward")
+
+
+def dz_chunk_attn_forward_noalloc(desc: dz_attn_desc, q, k, v, cache: Optional[dz_kvcache],
+                                  layout: dz_chunk_layout, out, stream=None) -> None:
+    """Attention for callers that cannot allocate device memory (no handle; static scratch)."""
+    cptr = ctypes.byref(cache) if cache is not None else None
+    _check(load().dz_chunk_attn_forward_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v),
+                                                cptr, ctypes.byref(layout), _ptr(out),
+                                                _stream(stream)),
+           "dz_chunk_attn_forward_noalloc")
 
 
 def dz_kvcache_append(handle: int, cache: dz_kvcache, k, v, stream=None) -> None:

@@ -194,6 +194,32 @@ dz_status dz_kvcache_append(dz_attn_t handle, dz_kvcache* cache, const void* k, 
 dz_status dz_kvcache_replace(dz_attn_t handle, dz_kvcache* cache, int32_t chunk_index,
                              const void* k, const void* v, void* stream);
 
+/* The same attention as dz_chunk_attn_forward, for callers that cannot call
+ * cudaMalloc: code that runs while a stream is being captured in global mode,
+ * runtimes that hand out device memory only from a pool they reserved up
+ * front, or plug-ins held to a fixed memory budget.  The paper has no
+ * counterpart; this is an interface choice of this library.
+ *
+ * It needs no handle and allocates nothing.  Its scratch memory (split
+ * results, split counters, a status word: 16.25 MiB) and its rotary tables
+ * (up to 294912 (cos, sin) entries, 2.25 MiB) are static device arrays of the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Limits (DZ_ERR_CAPACITY beyond them):
+ *   desc->max_batch * num_heads * ceil(desc->max_q_tokens / 256) * 2 <= 65536,
+ *   max_pos_t*pairs_t + max_pos_h*pairs_h + max_pos_w*pairs_w <= 294912;
+ * the split uses at most 63 CTAs, so large calls run slower than through a
+ * handle.  The first call on a device looks up the arrays' device addresses,
+ * and the first call with a given rotary configuration (base, pairs, max_pos)
+ * fills the tables with a synchronous copy: make those calls before any stream
+ * capture.  Every call clears the split counters on `stream` and then uses the
+ * same arrays, which keep the last call's contents: calls that overlap on the
+ * GPU (other streams, other threads) race and give wrong results.  Device-side
+ * timeouts are not reported on this path.  Arguments as dz_chunk_attn_forward,
+ * with desc in place of the handle. */
+dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* desc, const void* q, const void* k,
+                                        const void* v, const dz_kvcache* cache,
+                                        const dz_chunk_layout* layout, void* out, void* stream);
+
 /* Synchronise `stream`, read and clear the handle's device status word.
  * Returns DZ_ERR_TIMEOUT if a kernel's bounded wait ran out since the last
  * read, DZ_ERR_CUDA on a CUDA error, else DZ_OK. */
