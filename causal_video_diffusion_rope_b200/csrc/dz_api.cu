@@ -24,6 +24,8 @@ struct dz_attn {
   size_t n_counters;
   int* status;         // device status word
   PFN_cuTensorMapEncodeTiled_v12000 encode;
+  void* rot_ws;        // rotated q and k of teacher-forcing / prefill calls (or null)
+  int rot_tokens;      // query tokens per batch item rot_ws holds
 };
 
 namespace {
@@ -137,7 +139,7 @@ dz_status dz_attn_create(dz_attn_t* out, const dz_attn_desc* d) {
     return DZ_ERR_SHAPE;
   if (!(d->rope_base > 1.0) || !std::isfinite(d->rope_base)) return DZ_ERR_SHAPE;
   if (d->max_batch < 1 || d->max_q_tokens < 1 || d->max_pos_t < 1 || d->max_pos_h < 1 ||
-      d->max_pos_w < 1)
+      d->max_pos_w < 1 || d->prerotate_tokens < 0)
     return DZ_ERR_SHAPE;
   if (cdiv(d->max_q_tokens, dz::Q_GROUP) > dz::MAX_Q_GROUPS) return DZ_ERR_CAPACITY;
   if (static_cast<long long>(d->max_pos_t) * d->rope_pairs_t +
@@ -192,6 +194,13 @@ dz_status dz_attn_create(dz_attn_t* out, const dz_attn_desc* d) {
   if (e == cudaSuccess) e = cudaMalloc(&a->ws, ws_floats * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc(&a->counters, a->n_counters * sizeof(int));
   if (e == cudaSuccess) e = cudaMalloc(&a->status, sizeof(int));
+  a->rot_ws = nullptr;
+  a->rot_tokens = 0;
+  if (e == cudaSuccess && d->prerotate_tokens > 0) {
+    const size_t bytes = 2ull * d->max_batch * d->prerotate_tokens * d->num_heads * dz::HEAD_DIM * 2;
+    e = cudaMalloc(&a->rot_ws, bytes);
+    if (e == cudaSuccess) a->rot_tokens = d->prerotate_tokens;
+  }
   if (e == cudaSuccess)
     e = cudaMemcpy(a->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemset(a->counters, 0, a->n_counters * sizeof(int));
@@ -201,6 +210,7 @@ dz_status dz_attn_create(dz_attn_t* out, const dz_attn_desc* d) {
     cudaFree(a->ws);
     cudaFree(a->counters);
     cudaFree(a->status);
+    cudaFree(a->rot_ws);
     delete a;
     return DZ_ERR_CUDA;
   }
@@ -215,6 +225,7 @@ dz_status dz_attn_destroy(dz_attn_t a) {
   cudaFree(a->ws);
   cudaFree(a->counters);
   cudaFree(a->status);
+  cudaFree(a->rot_ws);
   delete a;
   return cuda_status(e);
 }
@@ -319,13 +330,31 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
                         static_cast<long long>(g.gw) * a->desc.rope_pairs_w;
     p.stage_ok = n <= dz::ROPE_STAGE_MAX ? 1 : 0;
   }
+  // teacher forcing / prefill: rotate q and k once into the workspace when it fits
+  const void* q_att = q;
+  const void* k_att = k;
+  if ((l->mode == DZ_MODE_TEACHER_FORCING || l->mode == DZ_MODE_PREFILL) && a->rot_ws &&
+      Sq <= a->rot_tokens && l->batch <= a->desc.max_batch) {
+    const size_t elems = static_cast<size_t>(l->batch) * Sq * H * dz::HEAD_DIM;
+    __nv_bfloat16* qr = static_cast<__nv_bfloat16*>(a->rot_ws);
+    __nv_bfloat16* kr = qr + elems;
+    const int period = l->mode == DZ_MODE_TEACHER_FORCING ? static_cast<int>(L * l->num_chunks) : 0;
+    st = cuda_status(dz::launch_rope3d(q, qr, l->batch, static_cast<int>(Sq), H, g, 0, tables_of(a),
+                                       static_cast<cudaStream_t>(stream), k, kr, period),
+                     "pre-rotation launch");
+    if (st != DZ_OK) return st;
+    q_att = qr;
+    k_att = kr;
+    p.rope_q = p.rope_k = 0;
+    p.stage_ok = 0;
+  }
   p.out = out;
   p.ws = a->ws;
   p.counters = a->counters;
   p.status = a->status;
 
-  st = make_map(a, &p.tm_q, q, l->batch, static_cast<int>(Sq), static_cast<int>(Sq), H);
-  if (st == DZ_OK) st = make_map(a, &p.tm_k, k, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
+  st = make_map(a, &p.tm_q, q_att, l->batch, static_cast<int>(Sq), static_cast<int>(Sq), H);
+  if (st == DZ_OK) st = make_map(a, &p.tm_k, k_att, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
   if (st == DZ_OK) st = make_map(a, &p.tm_v, v, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
   if (st == DZ_OK && cache_len > 0) {
     st = make_map(a, &p.tm_ck, cache->k, l->batch, cache_len, cache->capacity_tokens, H);
@@ -535,6 +564,8 @@ extern "C" dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* d, const 
   a.n_counters = static_cast<size_t>(d->max_batch) * d->num_heads * n_qg_max * dz::Q_TILES;
   a.status = reinterpret_cast<int*>(nd.scratch + NOALLOC_WS_BYTES + NOALLOC_COUNTERS * sizeof(int));
   a.encode = nd.encode;
+  a.rot_ws = nullptr;  // no pre-rotation workspace: rotation stays inside the kernel
+  a.rot_tokens = 0;
   // the split counters and the status word must start at zero (a previous call that
   // gave up may have left them set); cleared on the caller's stream
   cudaStream_t st = static_cast<cudaStream_t>(stream);

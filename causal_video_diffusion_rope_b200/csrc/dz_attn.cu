@@ -294,6 +294,44 @@ __device__ __forceinline__ float exp_pack(const uint32_t (&v)[32], uint32_t (&pk
   return (s4[0] + s4[1]) + (s4[2] + s4[3]);
 }
 
+// Rotate row r of a swizzled 128x128 bf16 tile (shared address `tile`) when the
+// pair split (PT, PH, PW) is known at compile time and the row's t-, h- and
+// w-table rows sit in shared memory at addresses tt, th, tw: every table read is
+// one shared load at a constant offset.
+template <int PT, int PH, int PW>
+__device__ __forceinline__ void rotate_tile_row_split(uint32_t tile, int r, uint32_t tt,
+                                                      uint32_t th, uint32_t tw) {
+  static_assert(PT + PH + PW == HEAD_DIM / 2, "pair split");
+  const uint32_t row = tile + r * 128;
+#pragma unroll
+  for (int b4 = 0; b4 < 4; ++b4) {
+    float2 cs[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int j = b4 * 16 + k;
+      cs[k] = lds_f2(j < PT ? tt + 8 * j : (j < PT + PH ? th + 8 * (j - PT) : tw + 8 * (j - PT - PH)));
+    }
+    uint4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = b4 * 4 + k;
+      v[k] = lds_u4(row + (c >> 3) * HALF_BYTES + (((c & 7) ^ (r & 7)) << 4));
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[k].x = rope_pair(v[k].x, cs[4 * k + 0]);
+      v[k].y = rope_pair(v[k].y, cs[4 * k + 1]);
+      v[k].z = rope_pair(v[k].z, cs[4 * k + 2]);
+      v[k].w = rope_pair(v[k].w, cs[4 * k + 3]);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int c = b4 * 4 + k;
+      sts_u4(row + (c >> 3) * HALF_BYTES + (((c & 7) ^ (r & 7)) << 4), v[k]);
+    }
+  }
+}
+
 __device__ __forceinline__ long long cta_start(long long c, long long W, int G) {
   return c * W / G;
 }
@@ -571,6 +609,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     // ======================= rotary gate =======================
     const int r0 = tid - WARP_ROPE * 32;  // rows r0 + k * ROPE_THREADS of a tile
+    // fast path: tables staged in shared memory and the 22/21/21 split
+    const bool fast = p.stage_ok && p.rope.pt == 22 && p.rope.ph == 21 && p.rope.pw == 21;
+    const uint32_t st_base = smem_u32(smem + SM_ROPE);
+    const uint32_t st_h = st_base + 8 * (p.stage_nt * 22);
+    const uint32_t st_w = st_h + 8 * (p.geom.gh * 21);
+    auto rotate_row = [&](uint8_t* tile, int r, int t, int h, int w) {
+      if (fast) {
+        rotate_tile_row_split<22, 21, 21>(smem_u32(tile), r, st_base + 8 * ((t - p.stage_t0) * 22),
+                                          st_h + 8 * (h * 21), st_w + 8 * (w * 21));
+      } else {
+        rotate_tile_row(tile, r, rope, t, h, w);
+      }
+    };
     long long pos = cstart;
     Seg sg;
     int seg_i = 0;
@@ -586,7 +637,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (s < p.sched.Sq) {
               int t, h, w;
               seq_pos(p, s, t, h, w);
-              rotate_tile_row(sQ + q * TILE_BYTES, r, rope, t, h, w);
+              rotate_row(sQ + q * TILE_BYTES, r, t, h, w);
             }
           }
         }
@@ -602,7 +653,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int r = r0; r < kt.nvalid; r += ROPE_THREADS) {
           int t, h, w;
           seq_pos(p, kt.row0 + r, t, h, w);
-          rotate_tile_row(sK + st * TILE_BYTES, r, rope, t, h, w);
+          rotate_row(sK + st * TILE_BYTES, r, t, h, w);
         }
         fence_proxy_async_smem();
         mbar_arrive(&bar[B_K_READY + st]);

@@ -157,8 +157,11 @@ __host__ __device__ __forceinline__ int unit_tile_count(const SchedGeom& g, int 
 cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int B, int rows,
                            int H, int cap, int dst_row0, cudaStream_t stream);
 
+// Rotates x into y (and x1 into y1 when x1 is not null) for B x S tokens; with
+// period > 0 token s is rotated at the position of token s % period.
 cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const ChunkGeom& g,
-                          int first_chunk, const RopeTables& r, cudaStream_t stream);
+                          int first_chunk, const RopeTables& r, cudaStream_t stream,
+                          const void* x1 = nullptr, void* y1 = nullptr, int period = 0);
 
 struct AttnLaunch {
   CUtensorMap tm_q, tm_k, tm_v, tm_ck, tm_cv;

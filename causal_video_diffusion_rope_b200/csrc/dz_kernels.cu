@@ -53,21 +53,25 @@ cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int
 }
 
 // ---------------------------------------------------------------------------
-// Standalone 3D rotary embedding.  One block per token (b, s): its position is
-// computed once; the block's threads rotate the token's H*16 16-byte chunks.
-// ---------------------------------------------------------------------------
+// 3D rotary embedding of whole tokens.  One block per token (b, s) of each of
+// up to two tensors (blockIdx.y): its position is computed once, then the
+// block's threads rotate the token's H*16 16-byte chunks.  With period > 0,
+// token s takes the position of token s % period (the noisy half of a
+// teacher-forcing sequence shares the clean half's positions).
 // x and y may be the same buffer (in place): each thread reads and then writes
 // the same 16 bytes, so they are not declared __restrict__.
-__global__ void __launch_bounds__(128) rope3d_kernel(const uint4* x, uint4* y, int S, int H,
-                                                     ChunkGeom g, int first_chunk,
-                                                     RopeTables r) {
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) rope3d_kernel(const uint4* x0, uint4* y0, const uint4* x1,
+                                                     uint4* y1, int S, int H, ChunkGeom g,
+                                                     int first_chunk, int period, RopeTables r) {
   const long long token = blockIdx.x;  // b * S + s
-  const int s = static_cast<int>(token % S);
+  int s = static_cast<int>(token % S);
+  if (period > 0) s %= period;
   int t, hh, w;
   token_pos(g, s, first_chunk, t, hh, w);
   const int nvec = H * (HEAD_DIM / 8);
-  const uint4* src = x + token * nvec;
-  uint4* dst = y + token * nvec;
+  const uint4* src = (blockIdx.y == 0 ? x0 : x1) + token * nvec;
+  uint4* dst = (blockIdx.y == 0 ? y0 : y1) + token * nvec;
   for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
     const int j0 = (i & 15) * 4;
     dst[i] = rope_chunk(src[i], r, j0, t, hh, w);
@@ -75,11 +79,14 @@ __global__ void __launch_bounds__(128) rope3d_kernel(const uint4* x, uint4* y, i
 }
 
 cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const ChunkGeom& g,
-                          int first_chunk, const RopeTables& r, cudaStream_t stream) {
+                          int first_chunk, const RopeTables& r, cudaStream_t stream,
+                          const void* x1, void* y1, int period) {
   const long long tokens = static_cast<long long>(B) * S;
   if (tokens <= 0) return cudaSuccess;
-  rope3d_kernel<<<static_cast<unsigned>(tokens), 128, 0, stream>>>(
-      static_cast<const uint4*>(x), static_cast<uint4*>(y), S, H, g, first_chunk, r);
+  dim3 grid(static_cast<unsigned>(tokens), x1 ? 2 : 1);
+  rope3d_kernel<<<grid, 128, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
+                                          static_cast<const uint4*>(x1), static_cast<uint4*>(y1),
+                                          S, H, g, first_chunk, period, r);
   return cudaGetLastError();
 }
 

@@ -51,7 +51,7 @@ class dz_attn_desc(ctypes.Structure):
         ("rope_pairs_w", ctypes.c_int32),
         ("max_batch", ctypes.c_int32), ("max_q_tokens", ctypes.c_int32),
         ("max_pos_t", ctypes.c_int32), ("max_pos_h", ctypes.c_int32),
-        ("max_pos_w", ctypes.c_int32),
+        ("max_pos_w", ctypes.c_int32), ("prerotate_tokens", ctypes.c_int32),
     ]
 
 
@@ -134,9 +134,10 @@ def _check(st: int, where: str) -> None:
 
 def make_desc(num_heads: int = 40, max_batch: int = 2, max_q_tokens: int = 8192,
               max_pos_t: int = 4096, max_pos_h: int = 256, max_pos_w: int = 256,
-              rope_base: float = 10000.0, pairs=(22, 21, 21)) -> dz_attn_desc:
+              rope_base: float = 10000.0, pairs=(22, 21, 21),
+              prerotate_tokens: int = 0) -> dz_attn_desc:
     return dz_attn_desc(num_heads, 128, rope_base, pairs[0], pairs[1], pairs[2], max_batch,
-                        max_q_tokens, max_pos_t, max_pos_h, max_pos_w)
+                        max_q_tokens, max_pos_t, max_pos_h, max_pos_w, prerotate_tokens)
 
 
 def make_layout(mode: int, batch: int, frames_per_chunk: int, grid_h: int, grid_w: int,

@@ -70,6 +70,14 @@ typedef struct dz_attn* dz_attn_t; /* opaque handle */
  *   max_pos_t/h/w      exclusive bounds of the (t, h, w) token positions the
  *                      rotary tables cover; a call whose tokens reach beyond
  *                      them returns DZ_ERR_SHAPE.
+ *   prerotate_tokens   0, or the largest query length (per batch item) of
+ *                      TEACHER_FORCING / PREFILL calls for which q and k are
+ *                      rotated once per call into a handle-owned workspace
+ *                      (2 * max_batch * prerotate_tokens * H * 256 bytes,
+ *                      allocated by dz_attn_create) before the attention runs;
+ *                      every key tile there is read by many query groups, so
+ *                      rotating it once is cheaper than rotating it on each
+ *                      load.  Other calls rotate inside the attention kernel.
  */
 typedef struct {
   int32_t num_heads;
@@ -79,6 +87,7 @@ typedef struct {
   int32_t max_batch;
   int32_t max_q_tokens;
   int32_t max_pos_t, max_pos_h, max_pos_w;
+  int32_t prerotate_tokens;
 } dz_attn_desc;
 
 typedef enum {

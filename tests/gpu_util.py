@@ -64,9 +64,10 @@ class Handle:
     """dz_attn handle for a given head count (destroyed on close)."""
 
     def __init__(self, heads: int, max_batch: int = 2, max_q_tokens: int = 16384,
-                 max_pos_t: int = 4096):
+                 max_pos_t: int = 4096, prerotate_tokens: int = 0):
         self.h = dz.dz_attn_create(dz.make_desc(num_heads=heads, max_batch=max_batch,
-                                                max_q_tokens=max_q_tokens, max_pos_t=max_pos_t))
+                                                max_q_tokens=max_q_tokens, max_pos_t=max_pos_t,
+                                                prerotate_tokens=prerotate_tokens))
         self.heads = heads
 
     def close(self):

@@ -31,10 +31,13 @@ def _cuda():
 _handles = {}
 
 
-def handle(heads):
-    if heads not in _handles:
-        _handles[heads] = Handle(heads)
-    return _handles[heads].h
+def handle(heads, prerotate=True):
+    """Handle for `heads`; with prerotate, teacher-forcing/prefill calls rotate q and k
+    once per call before the attention kernel, else the kernel rotates on each load."""
+    key = (heads, prerotate)
+    if key not in _handles:
+        _handles[key] = Handle(heads, prerotate_tokens=8192 if prerotate else 0)
+    return _handles[key].h
 
 
 def teardown_module(module):
@@ -47,8 +50,9 @@ def rand_bits(rng, shape, scale=1.0):
     return synth.bf16_bits_from_f32(rng.standard_normal(shape).astype(np.float32) * scale)
 
 
-def run_forward(lay: Layout, heads: int, q, k, v, cache_k=None, cache_v=None, cache_len=0):
-    h = handle(heads)
+def run_forward(lay: Layout, heads: int, q, k, v, cache_k=None, cache_v=None, cache_len=0,
+                prerotate=True):
+    h = handle(heads, prerotate)
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     cache = None
     keep = []
@@ -237,6 +241,22 @@ def test_attention_wide_scores(name, lay, heads, cache_len, scale):
     ref = oracle_full(lay, q, k, v, ck, cv, cache_len)
     assert_close(got, ref, name + " vs exact oracle", max_abs_tol=2e-2 * scale ** 2,
                  rel_tol=5e-3 * scale ** 2 / 4)
+
+
+FUSED_ROTATION_CASES = [c for c in SMALL_CASES if c[1].mode in (MODE_PREFILL, MODE_TEACHER_FORCING)]
+
+
+@pytest.mark.parametrize("name,lay,heads,cache_len,scale", FUSED_ROTATION_CASES,
+                         ids=[c[0] for c in FUSED_ROTATION_CASES])
+def test_attention_elementwise_rotation_in_kernel(name, lay, heads, cache_len, scale):
+    """Teacher forcing / prefill with the rotation done on each tile load (no workspace)."""
+    rng = np.random.default_rng(zlib.crc32(name.encode()) + 1)
+    B = lay.batch
+    q = rand_bits(rng, (B, lay.q_len, heads, D), scale)
+    k = rand_bits(rng, (B, lay.self_kv_len, heads, D), scale)
+    v = rand_bits(rng, (B, lay.self_kv_len, heads, D))
+    got = run_forward(lay, heads, q, k, v, prerotate=False)
+    assert_close(got, oracle_full(lay, q, k, v), name + " (rotation in kernel)")
 
 
 def test_single_visible_key_exact():
