@@ -35,7 +35,7 @@ from causal_video_diffusion_rope_b200 import synth  # noqa: E402
 
 METRIC = ("chunk-causal attn TFLOP/s and % of B200 BF16 peak; "
           "µs per DiT-layer attention call")
-WORKLOAD = synth.WORKLOADS[1]
+DEFAULT_WORKLOAD = 1  # single DiT-layer inference step
 L2_BYTES = 126 * 1024 * 1024
 KERNEL_SOURCES = ["causal_video_diffusion_rope_b200/csrc/dz_attn.cu",
                   "causal_video_diffusion_rope_b200/csrc/dz_internal.cuh",
@@ -59,15 +59,30 @@ def visible_pairs(w: synth.Workload) -> int:
 
 
 def step_flops(w: synth.Workload) -> float:
-    """Algorithmic FLOPs of one call: 4 * head_dim per visible pair per head per batch item."""
-    return 4.0 * w.head_dim * visible_pairs(w) * w.heads * w.layout.batch
+    """Algorithmic FLOPs of one step: 4 * head_dim per visible (query, key) pair per head per
+    batch item, for the self-attention call plus, in the long-cache workload, the
+    cross-attention call (every key visible)."""
+    f = 4.0 * w.head_dim * visible_pairs(w) * w.heads * w.layout.batch
+    if w.cross_kv_len:
+        f += 4.0 * w.head_dim * w.layout.chunk_len * w.cross_kv_len * w.heads * w.layout.batch
+    return f
 
 
 def step_bytes(w: synth.Workload) -> float:
-    """Bytes one call must move at least once: q, k, v, cached K/V, out (bf16)."""
+    """Bytes one step must move at least once: q, k, v, cached K/V, out (bf16), and the
+    cross-attention q, condition k/v and out."""
     lay = w.layout
     row = w.heads * w.head_dim * 2 * lay.batch
-    return row * (3 * lay.q_len + 2 * w.cache_tokens + lay.q_len)
+    n = 3 * lay.q_len + 2 * w.cache_tokens + lay.q_len
+    if w.cross_kv_len:
+        n += 2 * lay.chunk_len + 2 * w.cross_kv_len
+    return row * n
+
+
+def launches_per_step(w: synth.Workload) -> int:
+    """Kernels of this library one step launches: the once-per-call rotation of q and k and
+    the attention kernel, plus the cross-attention kernel in the long-cache workload."""
+    return 2 + (1 if w.cross_kv_len else 0)
 
 
 def sources_hash() -> str:
@@ -154,7 +169,7 @@ def oracle_rate(w: synth.Workload, inp, rng, budget_s: float, rows_per_call: int
     """
     from oracle import dz_oracle as O
     lay = w.layout
-    keys = w.cache_tokens + lay.chunk_len
+    keys = visible_pairs(w) / lay.q_len  # mean visible keys of a query row
     flops = 0.0
     calls = 0
     t0 = time.perf_counter()
@@ -163,8 +178,8 @@ def oracle_rate(w: synth.Workload, inp, rng, budget_s: float, rows_per_call: int
                  int(rng.integers(w.heads))) for _ in range(rows_per_call)]
         O.attention_rows(inp["q"], inp["k"], inp["v"], rows, lay.mode, lay.frames_per_chunk,
                          lay.grid_h, lay.grid_w, lay.n_action, lay.num_chunks,
-                         t_offset=lay.t_offset, cache_k_bits=inp["cache_k"],
-                         cache_v_bits=inp["cache_v"], cache_len=w.cache_tokens)
+                         t_offset=lay.t_offset, cache_k_bits=inp.get("cache_k"),
+                         cache_v_bits=inp.get("cache_v"), cache_len=w.cache_tokens)
         flops += 4.0 * w.head_dim * keys * rows_per_call
         calls += 1
         if time.perf_counter() - t0 >= budget_s:
@@ -195,14 +210,34 @@ def oracle_full_call_rate(w: synth.Workload, budget_s: float):
         h = heads_done % w.heads
         O.chunk_attn_forward(inp["q"], inp["k"], inp["v"], lay.mode, lay.frames_per_chunk,
                              lay.grid_h, lay.grid_w, lay.n_action, lay.num_chunks,
-                             t_offset=lay.t_offset, cache_k_bits=inp["cache_k"],
-                             cache_v_bits=inp["cache_v"], cache_len=w.cache_tokens,
+                             t_offset=lay.t_offset, cache_k_bits=inp.get("cache_k"),
+                             cache_v_bits=inp.get("cache_v"), cache_len=w.cache_tokens,
                              heads=slice(h, h + 4))
         heads_done += 4
         n += 1
     dt = time.perf_counter() - t0
-    flops = step_flops(w) / w.heads * heads_done
+    self_flops = 4.0 * w.head_dim * visible_pairs(w) * w.layout.batch
+    flops = self_flops * heads_done
     return flops / dt / 1e12, heads_done, dt
+
+
+# ----------------------------------------------------------------------------------- ranks
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time: every rank's elapsed milliseconds reduced with MAX."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOP/s: every rank runs `steps` independent calls (weak scaling);
+    the job takes as long as its slowest rank."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
 # ----------------------------------------------------------------------------------- GPU leg
@@ -214,27 +249,36 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = WORKLOAD
+    w = synth.WORKLOADS[args.workload]
     lay = w.layout
     B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
     per_set = step_bytes(w)
     n_sets = max(2, int(math.ceil(3 * L2_BYTES / per_set)))
-    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len))
+    # q and the chunk's own k are rotated once per call (prerotate_tokens) before the
+    # attention kernel; cache keys are stored rotated
+    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len,
+                                       prerotate_tokens=lay.q_len))
     dl = dz.layout_from(lay)
+    dlx = dz.layout_from(synth.cross_layout(w)) if w.cross_kv_len else None
     sets = []
     for i in range(n_sets):
         inp = synth.make_inputs(w, 1000 * rank + i)
         s = {k: torch.from_numpy(inp[k].view(np.int16)).to(dev).view(torch.bfloat16)
-             for k in ("q", "k", "v", "cache_k", "cache_v")}
-        s["out"] = torch.empty((B, L, H, D), dtype=torch.bfloat16, device=dev)
-        s["cache"] = dz.make_cache(s["cache_k"], s["cache_v"], B, w.cache_tokens,
-                                   w.cache_tokens, L)
+             for k in ("q", "k", "v", "cache_k", "cache_v", "q_x", "k_x", "v_x") if k in inp}
+        s["out"] = torch.empty((B, lay.q_len, H, D), dtype=torch.bfloat16, device=dev)
+        s["cache"] = (dz.make_cache(s["cache_k"], s["cache_v"], B, w.cache_tokens,
+                                    w.cache_tokens, L) if "cache_k" in s else None)
+        if w.cross_kv_len:
+            s["out_x"] = torch.empty((B, L, H, D), dtype=torch.bfloat16, device=dev)
         sets.append(s)
     stream = torch.cuda.Stream(device=dev)
 
     def call(i):
         s = sets[i % n_sets]
         dz.dz_chunk_attn_forward(h, s["q"], s["k"], s["v"], s["cache"], dl, s["out"], stream)
+        if dlx is not None:
+            dz.dz_chunk_attn_forward(h, s["q_x"], s["k_x"], s["v_x"], None, dlx, s["out_x"],
+                                     stream)
 
     # warm-up outside any graph
     with torch.cuda.stream(stream):
@@ -291,33 +335,30 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1)
     dz.dz_attn_sync_status(h, stream)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, dev)
     ms_per_step = ms / args.steps
     flops = step_flops(w)
-    tflops_total = flops * args.steps * world / (ms * 1e-3) / 1e12
+    tflops_total = job_throughput(flops, args.steps, world, ms)
 
-    # ---- end to end: host buffers in, result out, through the same C-ABI call
-    e2e = None
+    # ---- end to end: host buffers in, result out, through the same C-ABI calls
     s0 = sets[0]
-    hq = torch.empty_like(s0["q"], device="cpu").pin_memory()
-    hk = torch.empty_like(s0["k"], device="cpu").pin_memory()
-    hv = torch.empty_like(s0["v"], device="cpu").pin_memory()
-    ho = torch.empty_like(s0["out"], device="cpu").pin_memory()
-    hq.copy_(s0["q"].cpu())
-    hk.copy_(s0["k"].cpu())
-    hv.copy_(s0["v"].cpu())
-    dq, dk, dv = torch.empty_like(s0["q"]), torch.empty_like(s0["k"]), torch.empty_like(s0["v"])
+    in_keys = [k for k in ("q", "k", "v", "q_x", "k_x", "v_x") if k in s0]
+    out_keys = [k for k in ("out", "out_x") if k in s0]
+    host_in = {k: s0[k].cpu().pin_memory() for k in in_keys}
+    host_out = {k: torch.empty_like(s0[k], device="cpu").pin_memory() for k in out_keys}
+    dev_in = {k: torch.empty_like(s0[k]) for k in in_keys}
     n_e2e = max(3, min(args.steps, 200))
 
     def e2e_step():
-        dq.copy_(hq, non_blocking=True)
-        dk.copy_(hk, non_blocking=True)
-        dv.copy_(hv, non_blocking=True)
-        dz.dz_chunk_attn_forward(h, dq, dk, dv, s0["cache"], dl, s0["out"], stream)
-        ho.copy_(s0["out"], non_blocking=True)
+        for k in in_keys:
+            dev_in[k].copy_(host_in[k], non_blocking=True)
+        dz.dz_chunk_attn_forward(h, dev_in["q"], dev_in["k"], dev_in["v"], s0["cache"], dl,
+                                 s0["out"], stream)
+        if dlx is not None:
+            dz.dz_chunk_attn_forward(h, dev_in["q_x"], dev_in["k_x"], dev_in["v_x"], None, dlx,
+                                     s0["out_x"], stream)
+        for k in out_keys:
+            host_out[k].copy_(s0[k], non_blocking=True)
 
     with torch.cuda.stream(stream):
         for _ in range(3):
@@ -334,13 +375,11 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         x1.record(stream)
     stream.synchronize()
     ems = x0.elapsed_time(x1)
-    if world > 1:
-        t = torch.tensor([ems], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ems = float(t.item())
+    ems = max_over_ranks(ems, world, dev)
     dz.dz_attn_sync_status(h, stream)
-    e2e = {"value": round(flops * n_e2e * world / (ems * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
-           "h2d_bytes_per_step": int(hq.numel() * 2 * 3), "d2h_bytes_per_step": int(ho.numel() * 2),
+    e2e = {"value": round(job_throughput(flops, n_e2e, world, ems), 3), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(sum(host_in[k].numel() * 2 for k in in_keys)),
+           "d2h_bytes_per_step": int(sum(host_out[k].numel() * 2 for k in out_keys)),
            "ms_per_step": round(ems / n_e2e, 4), "steps": n_e2e}
 
     for gr in graphs.values():
@@ -358,6 +397,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle CPU work for the cpu_baseline field")
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
+                    choices=range(len(synth.WORKLOADS)),
+                    help="workload index (default: the single-layer inference step)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -365,11 +407,13 @@ def main():
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
-    w = WORKLOAD
+    w = synth.WORKLOADS[args.workload]
     config = {"workload": w.name, "batch": w.layout.batch, "heads": w.heads,
               "head_dim": w.head_dim, "q_tokens": w.layout.q_len,
-              "keys": w.cache_tokens + w.layout.chunk_len, "cache_tokens": w.cache_tokens,
-              "mode": "decode", "rope": "3d t/h/w 22/21/21 base 1e4 fused",
+              "keys": w.cache_tokens + w.layout.self_kv_len, "cache_tokens": w.cache_tokens,
+              "mode": synth.MODE_NAMES[w.layout.mode],
+              "cross_keys": w.cross_kv_len,
+              "rope": "3d t/h/w 22/21/21 base 1e4; q and the chunk's k rotated once per call",
               "flop_per_step": step_flops(w)}
 
     if args.impl == "reference":
@@ -441,7 +485,7 @@ def main():
                                       f"({n_sets * step_bytes(w) / 2**20:.0f} MiB > 126 MB L2)",
                            parallelism=f"dp{world} (independent replicas of the call)"),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clocks}
+            "gpu_launches": args.steps * launches_per_step(w), "clocks": clocks}
     print(json.dumps(line), flush=True)
 
 

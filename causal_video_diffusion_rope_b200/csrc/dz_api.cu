@@ -316,7 +316,23 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
   for (int qg = 0; qg < p.n_qg; ++qg) per_bh += dz::unit_tile_count(p.sched, qg);
   p.W = per_bh * l->batch * H;
   if (p.W <= 0) return DZ_ERR_SHAPE;
-  p.grid = static_cast<int>(p.W < a->num_sms ? p.W : a->num_sms);
+  // Work split: split units across CTAs (stream-K, with a merge of partial results)
+  // only when that shortens the longest CTA by more than the merge costs; a unit that
+  // one CTA runs whole writes its output directly.
+  {
+    const long long units = static_cast<long long>(l->batch) * H * p.n_qg;
+    int t_max = 0;
+    for (int qg = 0; qg < p.n_qg; ++qg) {
+      const int t = dz::unit_tile_count(p.sched, qg);
+      if (t > t_max) t_max = t;
+    }
+    const long long split_tiles = (p.W + a->num_sms - 1) / a->num_sms;
+    if (units <= a->num_sms && t_max <= split_tiles + dz::SPLIT_OVERHEAD_TILES) {
+      p.grid = static_cast<int>(units);
+    } else {
+      p.grid = static_cast<int>(p.W < a->num_sms ? p.W : a->num_sms);
+    }
+  }
   p.B = l->batch;
   p.H = H;
   p.geom = g;
@@ -330,17 +346,19 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
                         static_cast<long long>(g.gw) * a->desc.rope_pairs_w;
     p.stage_ok = n <= dz::ROPE_STAGE_MAX ? 1 : 0;
   }
-  // teacher forcing / prefill: rotate q and k once into the workspace when it fits
+  // with a workspace: rotate q and the call's own k once, before the attention kernel
   const void* q_att = q;
   const void* k_att = k;
-  if ((l->mode == DZ_MODE_TEACHER_FORCING || l->mode == DZ_MODE_PREFILL) && a->rot_ws &&
-      Sq <= a->rot_tokens && l->batch <= a->desc.max_batch) {
+  if (l->mode != DZ_MODE_CROSS && a->rot_ws && Sq <= a->rot_tokens &&
+      l->batch <= a->desc.max_batch) {
     const size_t elems = static_cast<size_t>(l->batch) * Sq * H * dz::HEAD_DIM;
     __nv_bfloat16* qr = static_cast<__nv_bfloat16*>(a->rot_ws);
     __nv_bfloat16* kr = qr + elems;
     const int period = l->mode == DZ_MODE_TEACHER_FORCING ? static_cast<int>(L * l->num_chunks) : 0;
-    st = cuda_status(dz::launch_rope3d(q, qr, l->batch, static_cast<int>(Sq), H, g, 0, tables_of(a),
-                                       static_cast<cudaStream_t>(stream), k, kr, period),
+    const int first = l->mode == DZ_MODE_DECODE ? l->num_chunks : 0;
+    st = cuda_status(dz::launch_rope3d(q, qr, l->batch, static_cast<int>(Sq), H, g, first,
+                                       tables_of(a), static_cast<cudaStream_t>(stream), k, kr,
+                                       period),
                      "pre-rotation launch");
     if (st != DZ_OK) return st;
     q_att = qr;

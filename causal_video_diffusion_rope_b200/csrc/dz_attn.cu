@@ -54,8 +54,8 @@ constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 // sub-partition); warpgroup 0 (producer, MMA, rotary) then gives registers to
 // the two softmax warpgroups.  The split must add up to the launch budget.
 constexpr int LAUNCH_REGS = 168;
-constexpr int REGS_CTRL = 104;
-constexpr int REGS_SOFT = 200;
+constexpr int REGS_CTRL = 136;
+constexpr int REGS_SOFT = 184;
 static_assert(REGS_CTRL + 2 * REGS_SOFT == 3 * LAUNCH_REGS, "register split must match launch");
 
 // shared memory layout (offsets from a 1024-byte aligned base)
@@ -280,18 +280,21 @@ __device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
 }
 
 // p = 2^(s * scale_log2 - mb) for 32 scores, packed as 16 bf16 pairs into pk[off, off + 16);
-// returns the fp32 sum of the 32 probabilities.
+// returns the fp32 sum of the 32 probabilities.  Pairs go through packed
+// two-lane fp32 FMA/add instructions.
 __device__ __forceinline__ float exp_pack(const uint32_t (&v)[32], uint32_t (&pk)[32], int off,
                                           float sl2, float mb) {
-  float s4[4] = {0.f, 0.f, 0.f, 0.f};
+  const float2 sc = make_float2(sl2, sl2), nm = make_float2(-mb, -mb);
+  float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const float p0 = ex2(__fmaf_rn(__uint_as_float(v[2 * j]), sl2, -mb));
-    const float p1 = ex2(__fmaf_rn(__uint_as_float(v[2 * j + 1]), sl2, -mb));
-    s4[j & 3] += p0 + p1;
-    pk[off + j] = pack_bf16x2(p0, p1);
+    const float2 x = ffma2(make_float2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])), sc, nm);
+    const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+    s2[j & 1] = fadd2(s2[j & 1], pp);
+    pk[off + j] = pack_bf16x2(pp.x, pp.y);
   }
-  return (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  const float2 t = fadd2(s2[0], s2[1]);
+  return t.x + t.y;
 }
 
 // Rotate row r of a swizzled 128x128 bf16 tile (shared address `tile`) when the
@@ -506,21 +509,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint32_t idesc_qk = idesc_bf16(TILE_M, TILE_N, false);
       const uint32_t idesc_pv = idesc_bf16(TILE_M, HEAD_DIM, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      // descriptors: only the low word (start address) changes between the K-steps
+      const uint32_t q_lo = desc_lo(sQa, 16), k_lo = desc_lo(sKa, 16), v_lo = desc_lo(sVa, HALF_BYTES);
       auto issue_qk = [&](int q, int st) {
-        const uint32_t a0 = sQa + q * TILE_BYTES, b0 = sKa + st * TILE_BYTES;
+        const uint32_t a0 = q_lo + ((q * TILE_BYTES) >> 4), b0 = k_lo + ((st * TILE_BYTES) >> 4);
+        const uint32_t d = tmem + q * TILE_N;
 #pragma unroll
         for (int kk = 0; kk < HEAD_DIM / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          mma_ss(tmem + q * TILE_N, smem_desc(a0 + off, 16, 1024), smem_desc(b0 + off, 16, 1024),
-                 idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+          mma_ss(d, desc_join(a0 + off), desc_join(b0 + off), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int q, int st, bool acc) {
-        const uint32_t b0 = sVa + st * TILE_BYTES;
+        const uint32_t b0 = v_lo + ((st * TILE_BYTES) >> 4);
+        const uint32_t d = tmem + 256 + q * HEAD_DIM, a = tmem + q * TILE_N;
 #pragma unroll
         for (int kk = 0; kk < TILE_N / 16; ++kk) {
-          mma_ts(tmem + 256 + q * HEAD_DIM, tmem + q * TILE_N + kk * 8,
-                 smem_desc(b0 + kk * 16 * 128, HALF_BYTES, 1024), idesc_pv,
+          mma_ts(d, a + kk * 8, desc_join(b0 + ((kk * 16 * 128) >> 4)), idesc_pv,
                  (acc || kk > 0) ? 1u : 0u);
         }
       };

@@ -182,6 +182,10 @@ struct AttnLaunch {
   int grid;
 };
 
+// Cost of splitting a unit across CTAs (partial write, merge, extra Q loads), in
+// key tiles: a call runs one unit per CTA unless splitting saves more than this.
+constexpr int SPLIT_OVERHEAD_TILES = 10;
+
 // Capacity (float2 entries) of the attention kernel's shared-memory rotary table.
 constexpr int ROPE_STAGE_MAX = 1280;
 

@@ -71,13 +71,14 @@ typedef struct dz_attn* dz_attn_t; /* opaque handle */
  *                      rotary tables cover; a call whose tokens reach beyond
  *                      them returns DZ_ERR_SHAPE.
  *   prerotate_tokens   0, or the largest query length (per batch item) of
- *                      TEACHER_FORCING / PREFILL calls for which q and k are
- *                      rotated once per call into a handle-owned workspace
- *                      (2 * max_batch * prerotate_tokens * H * 256 bytes,
- *                      allocated by dz_attn_create) before the attention runs;
- *                      every key tile there is read by many query groups, so
- *                      rotating it once is cheaper than rotating it on each
- *                      load.  Other calls rotate inside the attention kernel.
+ *                      DECODE / TEACHER_FORCING / PREFILL calls for which q and
+ *                      the call's own k are rotated once per call into a
+ *                      handle-owned workspace (2 * max_batch * prerotate_tokens
+ *                      * H * 256 bytes, allocated by dz_attn_create) before the
+ *                      attention kernel runs; a key tile is read by many query
+ *                      groups, so rotating it once is cheaper than rotating it
+ *                      on each load.  With 0 (or longer calls) the attention
+ *                      kernel rotates the tiles as it loads them.
  */
 typedef struct {
   int32_t num_heads;
