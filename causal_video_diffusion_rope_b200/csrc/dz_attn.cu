@@ -80,8 +80,7 @@ enum {
   B_P_FULL = B_S_FULL + Q_TILES,
   B_O_FULL = B_P_FULL + Q_TILES,
   B_O_FREE = B_O_FULL + Q_TILES,
-  B_WG = B_O_FREE + Q_TILES,       // softmax-group rendezvous (split combine)
-  B_DRAIN = B_WG + Q_TILES,
+  B_DRAIN = B_O_FREE + Q_TILES,
   B_COUNT = B_DRAIN + 1
 };
 constexpr int SM_MISC = SM_BAR + 256;         // tmem base, abort flag, combine flags
@@ -429,7 +428,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bar[B_P_FULL + q], 128);
       mbar_init(&bar[B_O_FULL + q], 1);
       mbar_init(&bar[B_O_FREE + q], 128);
-      mbar_init(&bar[B_WG + q], 128);
     }
     mbar_init(&bar[B_DRAIN], 1);
     *abort_flag = 0;
@@ -720,7 +718,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     long long pos = cstart;
     Seg sg;
     int seg_i = 0;
-    uint32_t tn = 0, wg_phase = 0;
+    uint32_t tn = 0;
     bool ok = true;
     while (ok && seg_next(p, prefix, pos, cend, sg)) {
       const int b = sg.bh / p.H, h = sg.bh - (sg.bh / p.H) * p.H;
@@ -825,119 +823,144 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           __syncwarp();
         }
       } else {
-        // partial piece: fp32 (O, m, l) to this CTA's slot, 16 columns at a time
-        const bool first_piece = cta_start(blockIdx.x, p.W, p.G) >= sg.u0;
-        const int slot = 2 * blockIdx.x + (first_piece ? 0 : 1);
-        float* buf = p.ws + static_cast<size_t>(slot) * PART_FLOATS;
-        float* obase = buf + static_cast<size_t>(q * TILE_M + 32 * quarter) * HEAD_DIM;
-#pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t v[16];
-          tmem_ld16(tO + c * 16, v);
-          tmem_wait_ld();
-          if (c == 7) {
-            tc_fence_before();
-            mbar_arrive(&bar[B_O_FREE + q]);
-          }
-          uint4* xrow = reinterpret_cast<uint4*>(xp + lane * XPOSE_PITCH);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) xrow[j] = make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-          __syncwarp();
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int task = lane + 32 * k;
-            const int rr = task >> 2, piece = task & 3;
-            const uint4 val = *reinterpret_cast<const uint4*>(xp + rr * XPOSE_PITCH + piece * 16);
-            *reinterpret_cast<uint4*>(obase + rr * HEAD_DIM + c * 16 + piece * 4) = val;
-          }
-          __syncwarp();
-        }
-        float* ml = buf + static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM;
-        reinterpret_cast<float2*>(ml)[q * TILE_M + r] = make_float2(m_run, l_run);
-        __threadfence();
-        mbar_arrive(&bar[B_WG + q]);
-        if (!mbar_wait(&bar[B_WG + q], wg_phase & 1, abort_flag, p.status)) break;
-        ++wg_phase;
+        // partial piece of a unit split across CTAs.  Its (bh, qg, q) counter
+        // counts arrivals in the low 16 bits and published partials in the high
+        // bits.  Every piece but the last to arrive publishes fp32 (O, m, l) in
+        // its slot; the last one waits for those and merges them with its own O,
+        // still in TMEM.  Slot layout: O as [32 column quads][Q_TILES * TILE_M
+        // rows] float4 (one warp access = 512 contiguous bytes), then (m, l) per
+        // row as float2.
+        constexpr int ROWS = Q_TILES * TILE_M;
+        const int row_l = q * TILE_M + r;
         const int c_first = cta_of(sg.u0, p.W, p.G);
         const int c_last = cta_of(sg.u1 - 1, p.W, p.G);
+        const int np = c_last - c_first + 1;
+        // slot of the piece held by CTA c: its first segment (slot 2c) unless the
+        // unit began before c's range, which only the first piece's CTA can see
+        const int slot0 = 2 * c_first + (cta_start(c_first, p.W, p.G) == sg.u0 ? 0 : 1);
+        const int me = static_cast<int>(blockIdx.x) - c_first;  // piece index
+        auto slot_of = [&](int k) { return k == 0 ? slot0 : 2 * (c_first + k); };
         int* counter = p.counters + (static_cast<size_t>(sg.bh) * p.n_qg + sg.qg) * Q_TILES + q;
         if (gtid == 0) {
           const int old = atomicAdd(counter, 1);
-          comb_flag[q] = (old == c_last - c_first) ? 1 : 0;
+          comb_flag[q] = ((old & 0xffff) == np - 1) ? 1 : 0;
         }
-        mbar_arrive(&bar[B_WG + q]);
-        if (!mbar_wait(&bar[B_WG + q], wg_phase & 1, abort_flag, p.status)) break;
-        ++wg_phase;
-        if (comb_flag[q]) {
-          // last piece to finish merges all pieces.  Lane = row for the (m, l) of
-          // every piece; then 4 rows at a time with lanes over the 128 columns, so
-          // the O loads of 4 rows x 4 pieces are in flight together and coalesced.
-          __threadfence();
-          const size_t ml_off = static_cast<size_t>(Q_TILES) * TILE_M * HEAD_DIM;
-          const int row_l = q * TILE_M + 32 * quarter + lane;  // this lane's row (m, l)
-          float M = -INFINITY;
-          for (int c2 = c_first; c2 <= c_last; ++c2) {
-            const int sl = 2 * c2 + (cta_start(c2, p.W, p.G) >= sg.u0 ? 0 : 1);
-            M = fmaxf(M, __ldcg(reinterpret_cast<const float2*>(p.ws + static_cast<size_t>(sl) * PART_FLOATS + ml_off) + row_l).x);
+        named_bar_sync(1 + q, 128);
+        // (both paths below pass another group barrier before comb_flag[q] can be rewritten)
+        const bool last = comb_flag[q] != 0;
+        if (!last) {
+          float4* o4 = reinterpret_cast<float4*>(p.ws + static_cast<size_t>(slot_of(me)) * PART_FLOATS);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
+            if (c == 3) {
+              tc_fence_before();
+              mbar_arrive(&bar[B_O_FREE + q]);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              o4[(c * 8 + j) * ROWS + row_l] =
+                  make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                              __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
           }
-          float Lsum = 0.f;
-          for (int c2 = c_first; c2 <= c_last; ++c2) {
-            const int sl = 2 * c2 + (cta_start(c2, p.W, p.G) >= sg.u0 ? 0 : 1);
-            const float2 ml2 = __ldcg(reinterpret_cast<const float2*>(p.ws + static_cast<size_t>(sl) * PART_FLOATS + ml_off) + row_l);
-            if (ml2.x != -INFINITY) Lsum += ml2.y * ex2(ml2.x - M);
+          reinterpret_cast<float2*>(p.ws + static_cast<size_t>(slot_of(me)) * PART_FLOATS +
+                                    static_cast<size_t>(ROWS) * HEAD_DIM)[row_l] =
+              make_float2(m_run, l_run);
+          __threadfence();
+          named_bar_sync(1 + q, 128);
+          if (gtid == 0) atomicAdd(counter, 1 << 16);
+        } else {
+          // wait until the other np - 1 pieces have published
+          if (gtid == 0) {
+            const int want = (np - 1) << 16;
+            const uint64_t t0 = globaltimer();
+            uint32_t n = 0;
+            while ((ld_acquire_gpu(counter) & ~0xffff) != want) {
+              if (((++n) & 63u) == 0u) {
+                if (*abort_flag) break;
+                if (globaltimer() - t0 > DZ_WAIT_NS) {
+                  *abort_flag = 1;
+                  atomicOr(p.status, DZ_DEV_TIMEOUT);
+                  break;
+                }
+              }
+            }
+          }
+          named_bar_sync(1 + q, 128);
+          if (*abort_flag) {
+            ok = false;
+            break;
+          }
+          __threadfence();
+          // merge the other pieces into this piece's O in TMEM, one piece per
+          // round trip (its (m, l) and whole row loaded together), rescaling
+          // online: O <- O * 2^(M - M') + O_k * 2^(m_k - M')
+          float M = m_run, Lsum = l_run;
+          for (int k = 0; k < np; ++k) {
+            if (k == me) continue;
+            const float* src = p.ws + static_cast<size_t>(slot_of(k)) * PART_FLOATS;
+            const float2 mk = __ldcg(reinterpret_cast<const float2*>(src + static_cast<size_t>(ROWS) * HEAD_DIM) + row_l);
+            float4 o[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __ldcg(reinterpret_cast<const float4*>(src) + j * ROWS + row_l);
+            // a row without visible keys in piece k leaves the row unchanged; the
+            // TMEM accesses below stay warp-uniform either way
+            const bool none = (mk.x == -INFINITY);
+            const float Mn = none ? M : fmaxf(M, mk.x);
+            const float a = none ? 1.f : ((M == -INFINITY) ? 0.f : ex2(M - Mn));
+            const float bk = none ? 0.f : ex2(mk.x - Mn);
+            Lsum = Lsum * a + mk.y * bk;
+            M = Mn;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              uint32_t v[32];
+              tmem_ld32(tO + g * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) * a + o[g * 8 + j].x * bk);
+                v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) * a + o[g * 8 + j].y * bk);
+                v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) * a + o[g * 8 + j].z * bk);
+                v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) * a + o[g * 8 + j].w * bk);
+              }
+              tmem_st32(tO + g * 32, v);
+            }
+            tmem_wait_st();
           }
           const float invL = 1.f / Lsum;
 #pragma unroll 1
-          for (int rr0 = 0; rr0 < 32; rr0 += 4) {
-            float4 acc[4];
-            float Mr[4], iL[4];
+          for (int g = 0; g < 4; ++g) {  // 32 output columns per pass
+            uint32_t v[32];
+            tmem_ld32(tO + g * 32, v);
+            tmem_wait_ld();
+            if (g == 3) {
+              tc_fence_before();
+              mbar_arrive(&bar[B_O_FREE + q]);
+            }
+            // bf16 row chunk through the warp's transpose buffer, then 64-byte row pieces
+            uint4* xrow = reinterpret_cast<uint4*>(xp + lane * XPOSE_PITCH);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              xrow[j] = make_uint4(
+                  pack_bf16x2(__uint_as_float(v[8 * j]) * invL, __uint_as_float(v[8 * j + 1]) * invL),
+                  pack_bf16x2(__uint_as_float(v[8 * j + 2]) * invL, __uint_as_float(v[8 * j + 3]) * invL),
+                  pack_bf16x2(__uint_as_float(v[8 * j + 4]) * invL, __uint_as_float(v[8 * j + 5]) * invL),
+                  pack_bf16x2(__uint_as_float(v[8 * j + 6]) * invL, __uint_as_float(v[8 * j + 7]) * invL));
+            __syncwarp();
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-              acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-              Mr[k] = __shfl_sync(0xffffffffu, M, rr0 + k);
-              iL[k] = __shfl_sync(0xffffffffu, invL, rr0 + k);
-            }
-            for (int c2 = c_first; c2 <= c_last; c2 += 4) {
-              float4 o[4][4];
-              float mm[4][4];
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int cc = c2 + u;
-                const int sl = 2 * cc + (cta_start(cc, p.W, p.G) >= sg.u0 ? 0 : 1);
-                const float* b2 = p.ws + static_cast<size_t>(sl) * PART_FLOATS;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const int row = q * TILE_M + 32 * quarter + rr0 + k;
-                  if (cc <= c_last) {
-                    mm[u][k] = __ldcg(reinterpret_cast<const float2*>(b2 + ml_off) + row).x;
-                    o[u][k] = __ldcg(reinterpret_cast<const float4*>(b2 + static_cast<size_t>(row) * HEAD_DIM) + lane);
-                  } else {
-                    mm[u][k] = -INFINITY;
-                    o[u][k] = make_float4(0.f, 0.f, 0.f, 0.f);
-                  }
-                }
-              }
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                  const float wgt = (mm[u][k] == -INFINITY) ? 0.f : ex2(mm[u][k] - Mr[k]);
-                  acc[k].x += wgt * o[u][k].x;
-                  acc[k].y += wgt * o[u][k].y;
-                  acc[k].z += wgt * o[u][k].z;
-                  acc[k].w += wgt * o[u][k].w;
-                }
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int s = row0 + rr0 + k;
+              const int task = lane + 32 * k;
+              const int rr = task >> 2, piece = task & 3;
+              const int s = row0 + rr;
+              const uint4 val = *reinterpret_cast<const uint4*>(xp + rr * XPOSE_PITCH + piece * 16);
               if (s < p.sched.Sq) {
-                __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + 4 * lane;
-                *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[k].x * iL[k], acc[k].y * iL[k]),
-                                                            pack_bf16x2(acc[k].z * iL[k], acc[k].w * iL[k]));
+                __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + g * 32 + piece * 8;
+                *reinterpret_cast<uint4*>(dst) = val;
               }
             }
+            __syncwarp();
           }
           if (gtid == 0) *counter = 0;  // ready for the next call
         }
