@@ -205,6 +205,9 @@ dz_status dz_attn_create(dz_attn_t* out, const dz_attn_desc* d) {
     e = cudaMemcpy(a->rope_tab, tab.data(), tab.size() * sizeof(float2), cudaMemcpyHostToDevice);
   if (e == cudaSuccess) e = cudaMemset(a->counters, 0, a->n_counters * sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(a->status, 0, sizeof(int));
+  // the copy and the memsets may return before they have landed; the handle's
+  // calls run on other streams
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
     cudaFree(a->rope_tab);
     cudaFree(a->ws);
@@ -333,6 +336,8 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
       p.grid = static_cast<int>(p.W < a->num_sms ? p.W : a->num_sms);
     }
   }
+  // the kernel schedules key tiles with 32-bit arithmetic
+  if (p.W * (p.grid + 1LL) >= (1LL << 31)) return DZ_ERR_UNSUPPORTED;
   p.B = l->batch;
   p.H = H;
   p.geom = g;
@@ -553,8 +558,9 @@ extern "C" dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* d, const 
         }
         off += static_cast<size_t>(npos[ax]) * npairs[ax];
       }
-      if (!tab.empty() && cudaMemcpy(nd.rope, tab.data(), tab.size() * sizeof(float2),
-                                     cudaMemcpyHostToDevice) != cudaSuccess)
+      if (!tab.empty() && (cudaMemcpy(nd.rope, tab.data(), tab.size() * sizeof(float2),
+                                      cudaMemcpyHostToDevice) != cudaSuccess ||
+                           cudaDeviceSynchronize() != cudaSuccess))
         return DZ_ERR_CUDA;
       nd.tables = true;
       nd.base = d->rope_base;

@@ -103,7 +103,7 @@ struct __align__(64) AttnParams {
   int B, H, n_qg;
   int rope_q, rope_k;
   int stage_ok, stage_t0, stage_nt;
-  long long W;
+  unsigned W;  // total key tiles; W * G < 2^31 (checked on the host)
   int G;
   float scale_log2;
 };
@@ -114,14 +114,14 @@ struct Seg {
   int t0, n;        // tile ordinals [t0, t0 + n) of the unit's list
   int e1, s2;       // the unit's list is [0, e1) then [s2, ...)
   bool full;        // this CTA covers the whole unit
-  long long u0, u1; // flattened tile range of the unit
+  unsigned u0, u1;  // flattened tile range of the unit
 };
 
-__device__ __forceinline__ bool seg_next(const AttnParams& p, const int* prefix, long long& pos,
-                                         long long end, Seg& s) {
+__device__ __forceinline__ bool seg_next(const AttnParams& p, const int* prefix, unsigned& pos,
+                                         unsigned end, Seg& s) {
   if (pos >= end) return false;
   const int Tbh = prefix[p.n_qg];
-  const long long bh = pos / Tbh;
+  const unsigned bh = pos / static_cast<unsigned>(Tbh);
   const int rem = static_cast<int>(pos - bh * Tbh);
   int lo = 0, hi = p.n_qg - 1;  // largest qg with prefix[qg] <= rem
   while (lo < hi) {
@@ -132,7 +132,7 @@ __device__ __forceinline__ bool seg_next(const AttnParams& p, const int* prefix,
   s.bh = static_cast<int>(bh);
   s.qg = lo;
   s.t0 = rem - prefix[lo];
-  long long seg_end = pos + (Tq - s.t0);
+  unsigned seg_end = pos + static_cast<unsigned>(Tq - s.t0);
   if (seg_end > end) seg_end = end;
   s.n = static_cast<int>(seg_end - pos);
   s.full = (s.t0 == 0 && s.n == Tq);
@@ -373,12 +373,12 @@ __device__ __forceinline__ void rotate_tile_row_split(uint32_t tile, int r, uint
   }
 }
 
-__device__ __forceinline__ long long cta_start(long long c, long long W, int G) {
-  return c * W / G;
+__device__ __forceinline__ unsigned cta_start(unsigned c, unsigned W, int G) {
+  return c * W / static_cast<unsigned>(G);
 }
 // The CTA whose range holds flattened tile x.
-__device__ __forceinline__ int cta_of(long long x, long long W, int G) {
-  return static_cast<int>(((x + 1) * G - 1) / W);
+__device__ __forceinline__ int cta_of(unsigned x, unsigned W, int G) {
+  return static_cast<int>(((x + 1) * static_cast<unsigned>(G) - 1) / W);
 }
 
 // Bounded wait that ignores the abort flag (used to drain in-flight copies).
@@ -432,6 +432,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bar[B_DRAIN], 1);
     *abort_flag = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&p.tm_q);
+    tma_prefetch_desc(&p.tm_k);
+    tma_prefetch_desc(&p.tm_v);
+    if (p.sched.nkc > 0) {
+      tma_prefetch_desc(&p.tm_ck);
+      tma_prefetch_desc(&p.tm_cv);
+    }
   }
   if (warp == WARP_MMA) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -474,22 +481,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const long long cstart = cta_start(blockIdx.x, p.W, p.G);
-  const long long cend = cta_start(blockIdx.x + 1, p.W, p.G);
+  const unsigned cstart = cta_start(blockIdx.x, p.W, p.G);
+  const unsigned cend = cta_start(blockIdx.x + 1, p.W, p.G);
 
   if (warp < WARP_SOFT) {
   regs_dec<REGS_CTRL>();
   if (warp == WARP_TMA) {
     // ======================= TMA producer =======================
     if (lane == 0) {
-      tma_prefetch_desc(&p.tm_q);
-      tma_prefetch_desc(&p.tm_k);
-      tma_prefetch_desc(&p.tm_v);
-      if (p.sched.nkc > 0) {
-        tma_prefetch_desc(&p.tm_ck);
-        tma_prefetch_desc(&p.tm_cv);
-      }
-      long long pos = cstart;
+      unsigned pos = cstart;
       Seg sg;
       int seg_i = 0;
       uint32_t k_iss = 0, v_iss = 0;  // K and V tiles issued so far
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  (acc || kk > 0) ? 1u : 0u);
         }
       };
-      long long pos = cstart;
+      unsigned pos = cstart;
       Seg sg;
       int seg_i = 0;
       uint32_t it = 0, tn = 0;
@@ -664,7 +664,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         rotate_tile_row(tile, r, rope, t, h, w);
       }
     };
-    long long pos = cstart;
+    unsigned pos = cstart;
     Seg sg;
     int seg_i = 0;
     uint32_t it = 0;
@@ -715,7 +715,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tO = tmem + lane_addr + 256 + q * HEAD_DIM;
     uint8_t* xp = smem + SM_X + (warp - WARP_SOFT) * XPOSE_WARP;  // this warp's transpose buffer
     const float sl2 = p.scale_log2;
-    long long pos = cstart;
+    unsigned pos = cstart;
     Seg sg;
     int seg_i = 0;
     uint32_t tn = 0;
@@ -1015,7 +1015,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   p.stage_ok = a.stage_ok;
   p.stage_t0 = a.stage_t0;
   p.stage_nt = a.stage_nt;
-  p.W = a.W;
+  p.W = static_cast<unsigned>(a.W);
   p.G = a.grid;
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));
   chunk_attn_kernel<<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);

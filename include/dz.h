@@ -177,7 +177,9 @@ dz_status dz_rope3d(dz_attn_t handle, const void* x, void* y, int32_t B, int32_t
  * bf16), softmax in fp32, probabilities rounded to bf16 for the PV product,
  * fp32 accumulation, output rounded to bf16.
  * Errors: DZ_ERR_INVALID_ARG, DZ_ERR_ALIGNMENT, DZ_ERR_SHAPE,
- * DZ_ERR_CAPACITY (batch or tokens beyond the handle), DZ_ERR_CUDA. */
+ * DZ_ERR_CAPACITY (batch or tokens beyond the handle), DZ_ERR_UNSUPPORTED
+ * (more than 2^31 / (SM count + 1) key tiles of 128 keys in one call),
+ * DZ_ERR_CUDA. */
 dz_status dz_chunk_attn_forward(dz_attn_t handle, const void* q, const void* k, const void* v,
                                 const dz_kvcache* cache, const dz_chunk_layout* layout,
                                 void* out, void* stream);
