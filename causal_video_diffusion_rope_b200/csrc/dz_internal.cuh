@@ -54,6 +54,9 @@ __device__ __forceinline__ int rope_index(const RopeTables& r, int j, int t, int
                   : (j < pth ? r.off_h + h * r.ph + (j - r.pt) : r.off_w + w * r.pw + (j - pth));
 }
 
+// One rotated pair (two bf16 in a 32-bit word) in fp32, rounded to bf16.  Used
+// by the standalone rotary kernel and the attention kernel's fused tile
+// rotation alike, so both give identical bf16 results.
 __device__ __forceinline__ uint32_t rope_pair(uint32_t xbits, float2 cs) {
   __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162*>(&xbits);
   const float x0 = __low2float(x), x1 = __high2float(x);
@@ -61,18 +64,6 @@ __device__ __forceinline__ uint32_t rope_pair(uint32_t xbits, float2 cs) {
   const float y1 = __fmaf_rn(x0, cs.y, __fmul_rn(x1, cs.x));
   __nv_bfloat162 y = __floats2bfloat162_rn(y0, y1);
   return *reinterpret_cast<uint32_t*>(&y);
-}
-
-// Rotate the 4 pairs (8 bf16) of one 16-byte chunk starting at pair j0.
-// Shared by the standalone rotary kernel and the attention kernel's fused
-// tile rotation, so both produce identical bf16 results.
-__device__ __forceinline__ uint4 rope_chunk(uint4 v, const RopeTables& r, int j0, int t, int h,
-                                            int w) {
-  v.x = rope_pair(v.x, __ldg(r.tab + rope_index(r, j0 + 0, t, h, w)));
-  v.y = rope_pair(v.y, __ldg(r.tab + rope_index(r, j0 + 1, t, h, w)));
-  v.z = rope_pair(v.z, __ldg(r.tab + rope_index(r, j0 + 2, t, h, w)));
-  v.w = rope_pair(v.w, __ldg(r.tab + rope_index(r, j0 + 3, t, h, w)));
-  return v;
 }
 
 // ---------------------------------------------------------------------------

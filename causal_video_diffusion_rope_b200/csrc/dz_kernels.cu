@@ -55,15 +55,22 @@ cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int
 // ---------------------------------------------------------------------------
 // 3D rotary embedding of whole tokens.  One block per token (b, s) of each of
 // up to two tensors (blockIdx.y): its position is computed once, then the
-// block's threads rotate the token's H*16 16-byte chunks.  With period > 0,
-// token s takes the position of token s % period (the noisy half of a
-// teacher-forcing sequence shares the clean half's positions).
+// block's threads rotate the token's H*16 16-byte chunks.  A thread always
+// handles the same 4 pairs (chunk index mod 16), so it reads its 4 (cos, sin)
+// entries once and then streams one chunk per head, all loads of a thread
+// issued before its stores.  With period > 0, token s takes the position of
+// token s % period (the noisy half of a teacher-forcing sequence shares the
+// clean half's positions).
 // x and y may be the same buffer (in place): each thread reads and then writes
 // the same 16 bytes, so they are not declared __restrict__.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) rope3d_kernel(const uint4* x0, uint4* y0, const uint4* x1,
-                                                     uint4* y1, int S, int H, ChunkGeom g,
-                                                     int first_chunk, int period, RopeTables r) {
+constexpr int ROPE_BLOCK = 128;
+constexpr int ROPE_UNROLL = 8;  // chunks per thread per pass: 64 heads with 128 threads
+
+__global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, uint4* y0,
+                                                            const uint4* x1, uint4* y1, int S,
+                                                            int H, ChunkGeom g, int first_chunk,
+                                                            int period, RopeTables r) {
   const long long token = blockIdx.x;  // b * S + s
   int s = static_cast<int>(token % S);
   if (period > 0) s %= period;
@@ -72,9 +79,24 @@ __global__ void __launch_bounds__(128) rope3d_kernel(const uint4* x0, uint4* y0,
   const int nvec = H * (HEAD_DIM / 8);
   const uint4* src = (blockIdx.y == 0 ? x0 : x1) + token * nvec;
   uint4* dst = (blockIdx.y == 0 ? y0 : y1) + token * nvec;
-  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-    const int j0 = (i & 15) * 4;
-    dst[i] = rope_chunk(src[i], r, j0, t, hh, w);
+  const int j0 = (threadIdx.x & 15) * 4;  // ROPE_BLOCK is a multiple of 16
+  float2 cs[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) cs[k] = __ldg(r.tab + rope_index(r, j0 + k, t, hh, w));
+  for (int i0 = threadIdx.x; i0 < nvec; i0 += ROPE_BLOCK * ROPE_UNROLL) {
+    uint4 v[ROPE_UNROLL];
+#pragma unroll
+    for (int u = 0; u < ROPE_UNROLL; ++u) {
+      const int i = i0 + u * ROPE_BLOCK;
+      if (i < nvec) v[u] = src[i];
+    }
+#pragma unroll
+    for (int u = 0; u < ROPE_UNROLL; ++u) {
+      const int i = i0 + u * ROPE_BLOCK;
+      if (i < nvec)
+        dst[i] = make_uint4(rope_pair(v[u].x, cs[0]), rope_pair(v[u].y, cs[1]),
+                            rope_pair(v[u].z, cs[2]), rope_pair(v[u].w, cs[3]));
+    }
   }
 }
 
@@ -84,7 +106,7 @@ cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const Chu
   const long long tokens = static_cast<long long>(B) * S;
   if (tokens <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(tokens), x1 ? 2 : 1);
-  rope3d_kernel<<<grid, 128, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
+  rope3d_kernel<<<grid, ROPE_BLOCK, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
                                           static_cast<const uint4*>(x1), static_cast<uint4*>(y1),
                                           S, H, g, first_chunk, period, r);
   return cudaGetLastError();
