@@ -255,6 +255,11 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
                                 const dz_kvcache* cache, const dz_chunk_layout* l, void* out,
                                 void* stream) {
   if (!a || !q || !k || !v || !l || !out) return DZ_ERR_INVALID_ARG;
+  // inputs already rotated: the flag is taken off a local copy of the layout
+  const bool given_rotated = (l->mode & DZ_MODE_ROTATED) != 0;
+  dz_chunk_layout l_plain = *l;
+  l_plain.mode &= ~DZ_MODE_ROTATED;
+  l = &l_plain;
   if (l->mode < DZ_MODE_DECODE || l->mode > DZ_MODE_CROSS) return DZ_ERR_INVALID_ARG;
   dz_status st = check_geom(l);
   if (st != DZ_OK) return st;
@@ -342,7 +347,7 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
   p.H = H;
   p.geom = g;
   p.rope = tables_of(a);
-  p.rope_q = p.rope_k = (l->mode != DZ_MODE_CROSS) ? 1 : 0;
+  p.rope_q = p.rope_k = (l->mode != DZ_MODE_CROSS && !given_rotated) ? 1 : 0;
   if (p.rope_q) {
     p.stage_t0 = g.t_offset + (l->mode == DZ_MODE_DECODE ? l->num_chunks * g.F : 0);
     p.stage_nt = (l->mode == DZ_MODE_DECODE ? 1 : l->num_chunks) * g.F;
@@ -354,7 +359,7 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
   // with a workspace: rotate q and the call's own k once, before the attention kernel
   const void* q_att = q;
   const void* k_att = k;
-  if (l->mode != DZ_MODE_CROSS && a->rot_ws && Sq <= a->rot_tokens &&
+  if (p.rope_q && a->rot_ws && Sq <= a->rot_tokens &&
       l->batch <= a->desc.max_batch) {
     const size_t elems = static_cast<size_t>(l->batch) * Sq * H * dz::HEAD_DIM;
     __nv_bfloat16* qr = static_cast<__nv_bfloat16*>(a->rot_ws);
@@ -421,6 +426,72 @@ dz_status dz_kvcache_replace(dz_attn_t a, dz_kvcache* c, int32_t chunk_index, co
                                         a->desc.num_heads, c->capacity_tokens,
                                         chunk_index * c->chunk_len,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int32_t S,
+                      int32_t d_model, const dz_chunk_layout* l, int32_t first_chunk,
+                      void* q_out, void* k_out, void* v_out, dz_kvcache* cache, void* stream) {
+  if (!a || !x || !w || !l || !q_out || !k_out || !v_out) return DZ_ERR_INVALID_ARG;
+  if (B < 1 || S < 1 || first_chunk < 0) return DZ_ERR_INVALID_ARG;
+  dz_status st = check_geom(l);
+  if (st != DZ_OK) return st;
+  if (d_model < 64 || d_model % 64 != 0) return DZ_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(q_out) || !aligned16(k_out) ||
+      !aligned16(v_out))
+    return DZ_ERR_ALIGNMENT;
+  if (B > a->desc.max_batch) return DZ_ERR_CAPACITY;
+  const int H = a->desc.num_heads;
+  const long long M = static_cast<long long>(B) * S;
+  const long long N = 3LL * H * dz::HEAD_DIM;
+  if (M >= (1LL << 31) / dz::HEAD_DIM || N >= (1LL << 31)) return DZ_ERR_SHAPE;
+  const dz::ChunkGeom g = geom_of(l);
+  st = check_positions(a, g, first_chunk, first_chunk + (S - 1) / g.L);
+  if (st != DZ_OK) return st;
+  dz::QkvLaunch p = {};
+  if (cache) {
+    if (!cache->k || !cache->v) return DZ_ERR_INVALID_ARG;
+    if (!aligned16(cache->k) || !aligned16(cache->v)) return DZ_ERR_ALIGNMENT;
+    if (cache->batch != B || cache->chunk_len != S || cache->len_tokens < 0 ||
+        cache->len_tokens > cache->capacity_tokens)
+      return DZ_ERR_INVALID_ARG;
+    if (static_cast<long long>(cache->len_tokens) + S > cache->capacity_tokens)
+      return DZ_ERR_CAPACITY;
+    p.ck = cache->k;
+    p.cv = cache->v;
+    p.cache_cap = cache->capacity_tokens;
+    p.cache_row0 = cache->len_tokens;
+  }
+  // x as [M][d_model] with 64 x 128 boxes, w as [N][d_model] with 64 x 256 boxes
+  auto map2d = [&](CUtensorMap* m, const void* base, long long rows, int box_rows) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d_model) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = a->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                                 dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? DZ_OK : DZ_ERR_CUDA;
+  };
+  st = map2d(&p.tm_x, x, M, 128);
+  if (st == DZ_OK) st = map2d(&p.tm_w, w, N, 256);
+  if (st != DZ_OK) return st;
+  p.q = q_out;
+  p.k = k_out;
+  p.v = v_out;
+  p.M = static_cast<int>(M);
+  p.S = S;
+  p.H = H;
+  p.K = d_model;
+  p.rope = tables_of(a);
+  p.geom = g;
+  p.first_chunk = first_chunk;
+  p.status = a->status;
+  p.num_sms = a->num_sms;
+  st = cuda_status(dz::launch_qkv_rope(p, static_cast<cudaStream_t>(stream)), "qkv launch");
+  if (st != DZ_OK) return st;
+  if (cache) cache->len_tokens += S;
+  return DZ_OK;
 }
 
 dz_status dz_attn_sync_status(dz_attn_t a, void* stream) {

@@ -182,6 +182,21 @@ constexpr int ROPE_STAGE_MAX = 1280;
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
 
+// Fused QKV projection + rotation (+ cache append); see dz_qkv.cu.
+struct QkvLaunch {
+  CUtensorMap tm_x, tm_w;  // x [M][K], w [3*H*128][K], bf16, 64 x (128 | 256) boxes, SW128
+  void *q, *k, *v;         // [M][H][128]
+  void *ck, *cv;           // cache or null
+  int cache_cap, cache_row0;
+  int M, S, H, K;
+  RopeTables rope;
+  ChunkGeom geom;
+  int first_chunk;
+  int* status;
+  int num_sms;
+};
+cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream);
+
 // Workspace (in floats) one partial-result slot needs: Q_TILES * TILE_M rows of
 // HEAD_DIM accumulators plus (m, l) per row.
 constexpr size_t PART_FLOATS = static_cast<size_t>(Q_TILES) * TILE_M * (HEAD_DIM + 2);

@@ -1,0 +1,276 @@
+// QKV projection of a run of chunk tokens with the 3D rotary embedding and the
+// KV-cache append fused into the GEMM epilogue.
+//
+// y = x W^T for x bf16 [M][K] (M = B*S tokens, K = d_model) and W bf16 [N][K]
+// (N = 3*H*128 output features: q, then k, then v, each head's 128 features
+// contiguous).  The q and k features of every token are turned by the token's
+// (t, h, w) rotation in fp32 straight from the fp32 accumulator, then every
+// output is rounded once to bf16 and written as q, k, v [M][H][128]; with a
+// cache, k and v also go to cache rows [row0, row0 + S) of their batch item.
+// The projection is the causal self-attention's input step in the DiT block
+// ("DreamZero (WAM) 模型架构", §2.3 block diagram: RMSNorm, modulation, causal
+// self-attention with RoPE on the latent sequence).
+//
+// One persistent CTA per SM walks output tiles of 128 tokens x 256 features
+// (two heads), n-tile major so that the CTAs working at one time share the
+// same weight tile through L2.  Warp 0 issues TMA loads of 64-wide K slices
+// into a 4-stage ring, warp 1 allocates TMEM and issues tcgen05.mma (M=128,
+// N=256, K=16, both operands K-major SW128 in shared memory), accumulating in
+// one of two 256-column TMEM buffers, and warps 2-5 drain the other buffer
+// (rotation, bf16 rounding, stores) while the next tile accumulates.
+#include "dz_internal.cuh"
+#include "dz_ptx.cuh"
+
+namespace dz {
+
+namespace {
+
+constexpr int QBM = 128, QBN = 256, QBK = 64, QSTAGES = 4;
+constexpr int QTHREADS = 192;
+constexpr int QA_BYTES = QBM * QBK * 2;  // 16 KiB
+constexpr int QB_BYTES = QBN * QBK * 2;  // 32 KiB
+constexpr int QSTAGE_BYTES = QA_BYTES + QB_BYTES;
+constexpr int QSM_BAR = QSTAGES * QSTAGE_BYTES;
+constexpr int QSM_MISC = QSM_BAR + 256;
+constexpr int QSMEM_BYTES = QSM_MISC + 64 + 1024;  // + alignment slack
+static_assert(QSMEM_BYTES <= 232448, "shared memory");
+
+enum {
+  QB_FULL = 0,
+  QB_EMPTY = QB_FULL + QSTAGES,
+  QB_ACC_FULL = QB_EMPTY + QSTAGES,
+  QB_ACC_EMPTY = QB_ACC_FULL + 2,
+  QB_DRAIN = QB_ACC_EMPTY + 2,
+  QB_COUNT = QB_DRAIN + 1
+};
+static_assert(QB_COUNT * 8 <= 256, "barrier area");
+
+struct __align__(64) QkvParams {
+  CUtensorMap tm_x, tm_w;
+  __nv_bfloat16 *q, *k, *v;
+  __nv_bfloat16 *ck, *cv;  // cache (null: no append)
+  int cache_cap, cache_row0;
+  int M, S, H, K, N;
+  int m_tiles, n_tiles;
+  RopeTables rope;
+  ChunkGeom geom;
+  int first_chunk;
+  int* status;
+};
+
+// 16 B stores of 32 bf16 values (a 64-byte row piece).
+__device__ __forceinline__ void store_piece(__nv_bfloat16* dst, const uint32_t (&pk)[16]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) d[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+}
+
+__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer() - t0 > DZ_WAIT_NS) return;
+  }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_constant__ QkvParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + QSM_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + QSM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + QSM_MISC + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int total = p.m_tiles * p.n_tiles;
+  const int KB = p.K / QBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < QSTAGES; ++s) {
+      mbar_init(&bar[QB_FULL + s], 1);
+      mbar_init(&bar[QB_EMPTY + s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar[QB_ACC_FULL + b], 1);
+      mbar_init(&bar[QB_ACC_EMPTY + b], 128);
+    }
+    mbar_init(&bar[QB_DRAIN], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&p.tm_x);
+    tma_prefetch_desc(&p.tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        const int nt = tile / p.m_tiles, mt = tile - nt * p.m_tiles;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int st = it % QSTAGES;
+          const uint32_t ph = (it / QSTAGES) & 1;
+          if (!mbar_wait(&bar[QB_EMPTY + st], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+          uint8_t* sa = smem + st * QSTAGE_BYTES;
+          mbar_expect_tx(&bar[QB_FULL + st], QSTAGE_BYTES);
+          tma_load_2d(sa, &p.tm_x, &bar[QB_FULL + st], kb * QBK, mt * QBM);
+          tma_load_2d(sa + QA_BYTES, &p.tm_w, &bar[QB_FULL + st], kb * QBK, nt * QBN);
+        }
+      }
+      // every issued copy has landed before the CTA exits
+      const uint32_t n_iss = it;
+      for (uint32_t j = (n_iss > QSTAGES ? n_iss - QSTAGES : 0); j < n_iss; ++j)
+        drain(&bar[QB_FULL + j % QSTAGES], (j / QSTAGES) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------- tcgen05 issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(QBM, QBN, false);
+      const uint32_t base_lo = desc_lo(smem_u32(smem), 16);
+      uint32_t it = 0;
+      int lt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        // the epilogue has drained this buffer (tile lt - 2)
+        if (!mbar_wait(&bar[QB_ACC_EMPTY + buf], ((lt >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * QBN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int st = it % QSTAGES;
+          const uint32_t ph = (it / QSTAGES) & 1;
+          if (!mbar_wait(&bar[QB_FULL + st], ph, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = base_lo + ((st * QSTAGE_BYTES) >> 4);
+          const uint32_t b0 = a0 + (QA_BYTES >> 4);
+#pragma unroll
+          for (int kk = 0; kk < QBK / 16; ++kk)
+            mma_ss(d, desc_join(a0 + ((kk * 32) >> 4)), desc_join(b0 + ((kk * 32) >> 4)), idesc,
+                   (kb > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&bar[QB_EMPTY + st]);
+        }
+        if (!ok) break;
+        mma_commit(&bar[QB_ACC_FULL + buf]);
+      }
+      mma_commit(&bar[QB_DRAIN]);
+      drain(&bar[QB_DRAIN], 0);
+    }
+  } else {
+    // ---------------- epilogue: warps 2..5, one token row per thread ----------------
+    const int quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
+    const int HD = p.H * HEAD_DIM;
+    int lt = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
+      const int buf = lt & 1;
+      if (!mbar_wait(&bar[QB_ACC_FULL + buf], (lt >> 1) & 1, abort_flag, p.status)) break;
+      tc_fence_after();
+      const int nt = tile / p.m_tiles, mt = tile - nt * p.m_tiles;
+      const int m = mt * QBM + r;
+      const bool valid = m < p.M;
+      const int bb = valid ? m / p.S : 0;
+      const int s = valid ? m - bb * p.S : 0;
+      int t = 0, hh = 0, w = 0;
+      token_pos(p.geom, s, p.first_chunk, t, hh, w);
+#pragma unroll 1
+      for (int c = 0; c < QBN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_addr + buf * QBN + c * 32, v);
+        tmem_wait_ld();
+        if (c == QBN / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&bar[QB_ACC_EMPTY + buf]);
+        }
+        const int n = nt * QBN + c * 32;  // feature of column 0 of this piece
+        if (n >= p.N) continue;
+        const int sec = n / HD;  // 0 q, 1 k, 2 v
+        const int rem = n - sec * HD;
+        const int head = rem / HEAD_DIM, d0 = rem - head * HEAD_DIM;
+        uint32_t pk[16];
+        if (sec < 2) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 cs = __ldg(p.rope.tab + rope_index(p.rope, (d0 >> 1) + i, t, hh, w));
+            const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
+            const float y0 = __fmaf_rn(x0, cs.x, -__fmul_rn(x1, cs.y));
+            const float y1 = __fmaf_rn(x0, cs.y, __fmul_rn(x1, cs.x));
+            pk[i] = pack_bf16x2(y0, y1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        if (valid) {
+          __nv_bfloat16* dst = (sec == 0 ? p.q : (sec == 1 ? p.k : p.v)) +
+                               (static_cast<size_t>(m) * p.H + head) * HEAD_DIM + d0;
+          store_piece(dst, pk);
+          if (sec > 0 && p.ck) {
+            __nv_bfloat16* cdst = (sec == 1 ? p.ck : p.cv) +
+                                  ((static_cast<size_t>(bb) * p.cache_cap + p.cache_row0 + s) * p.H + head) *
+                                      HEAD_DIM + d0;
+            store_piece(cdst, pk);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        qkv_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, QSMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  QkvParams p;
+  p.tm_x = a.tm_x;
+  p.tm_w = a.tm_w;
+  p.q = static_cast<__nv_bfloat16*>(a.q);
+  p.k = static_cast<__nv_bfloat16*>(a.k);
+  p.v = static_cast<__nv_bfloat16*>(a.v);
+  p.ck = static_cast<__nv_bfloat16*>(a.ck);
+  p.cv = static_cast<__nv_bfloat16*>(a.cv);
+  p.cache_cap = a.cache_cap;
+  p.cache_row0 = a.cache_row0;
+  p.M = a.M;
+  p.S = a.S;
+  p.H = a.H;
+  p.K = a.K;
+  p.N = 3 * a.H * HEAD_DIM;
+  p.m_tiles = (a.M + QBM - 1) / QBM;
+  p.n_tiles = (p.N + QBN - 1) / QBN;
+  p.rope = a.rope;
+  p.geom = a.geom;
+  p.first_chunk = a.first_chunk;
+  p.status = a.status;
+  const int total = p.m_tiles * p.n_tiles;
+  const int grid = total < a.num_sms ? total : a.num_sms;
+  qkv_rope_kernel<<<grid, QTHREADS, QSMEM_BYTES, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace dz

@@ -28,12 +28,13 @@ DZ_MODE_DECODE = 0
 DZ_MODE_TEACHER_FORCING = 1
 DZ_MODE_PREFILL = 2
 DZ_MODE_CROSS = 3
+DZ_MODE_ROTATED = 0x100  # flag: q and the call's own k are already rotated
 
 # Every entry point include/dz.h declares.
 EXPORTS = [
     "dz_attn_create", "dz_attn_destroy", "dz_rope3d", "dz_chunk_attn_forward",
     "dz_kvcache_append", "dz_kvcache_replace", "dz_attn_sync_status", "dz_status_string",
-    "dz_chunk_attn_forward_noalloc",
+    "dz_chunk_attn_forward_noalloc", "dz_qkv_rope",
 ]
 
 
@@ -96,6 +97,8 @@ def load() -> ctypes.CDLL:
         ctypes.POINTER(dz_chunk_layout), vp, vp]
     lib.dz_kvcache_append.argtypes = [vp, ctypes.POINTER(dz_kvcache), vp, vp, vp]
     lib.dz_kvcache_replace.argtypes = [vp, ctypes.POINTER(dz_kvcache), i32, vp, vp, vp]
+    lib.dz_qkv_rope.argtypes = [vp, vp, vp, i32, i32, i32, ctypes.POINTER(dz_chunk_layout), i32,
+                                vp, vp, vp, ctypes.POINTER(dz_kvcache), vp]
     lib.dz_attn_sync_status.argtypes = [vp, vp]
     lib.dz_status_string.argtypes = [ctypes.c_int]
     lib.dz_status_string.restype = ctypes.c_char_p
@@ -203,6 +206,16 @@ def dz_kvcache_replace(handle: int, cache: dz_kvcache, chunk_index: int, k, v,
                        stream=None) -> None:
     _check(load().dz_kvcache_replace(handle, ctypes.byref(cache), chunk_index, _ptr(k), _ptr(v),
                                      _stream(stream)), "dz_kvcache_replace")
+
+
+def dz_qkv_rope(handle: int, x, w, B: int, S: int, d_model: int, layout: dz_chunk_layout,
+                first_chunk: int, q_out, k_out, v_out, cache: Optional[dz_kvcache] = None,
+                stream=None) -> None:
+    """QKV projection with the rotation (and optionally the cache append) fused in."""
+    cptr = ctypes.byref(cache) if cache is not None else None
+    _check(load().dz_qkv_rope(handle, _ptr(x), _ptr(w), B, S, d_model, ctypes.byref(layout),
+                              first_chunk, _ptr(q_out), _ptr(k_out), _ptr(v_out), cptr,
+                              _stream(stream)), "dz_qkv_rope")
 
 
 def dz_attn_sync_status(handle: int, stream=None) -> None:

@@ -119,6 +119,13 @@ WORKLOADS = [
         cache_tokens=32 * 464, cross_kv_len=512 + 257, k_boost=3.0, k_boost_frac=0.05,
         description="cache of 32 chunks (15312 keys incl. self) + cross-attention to "
                     "512 text + 257 image keys; K x3 on 5% of heads"),
+    Workload(
+        "decode_b1_h40_3view_q1784_cache4", heads=40,
+        layout=Layout(MODE_DECODE, batch=1, frames_per_chunk=2, grid_h=22, grid_w=40,
+                      n_action=24, num_chunks=4),
+        cache_tokens=4 * 1784,
+        description="three camera views tiled to 352x640 (22x40 = 880 tokens per latent "
+                    "frame): 1784-token chunk over a cache of 4 chunks + itself (8920 keys)"),
 ]
 
 
@@ -156,6 +163,17 @@ def boosted_heads(rng: np.random.Generator, heads: int, frac: float) -> np.ndarr
     if n == 0:
         return np.zeros(0, dtype=np.int64)
     return np.sort(rng.choice(heads, size=n, replace=False))
+
+
+def projection_inputs(seed: int, B: int, S: int, d_model: int, heads: int, head_dim: int = 128):
+    """Hidden states x [B, S, d_model] ~ N(0, 1) and projection weights
+    w [3 * heads * head_dim, d_model] ~ N(0, 1 / d_model) (random init: no trained
+    weights), both drawn in fp32 and rounded to bf16; returns uint16 bit arrays."""
+    rng = np.random.default_rng(seed)
+    x = bf16_bits_from_f32(rng.standard_normal((B, S, d_model), dtype=np.float32))
+    w = bf16_bits_from_f32(rng.standard_normal((3 * heads * head_dim, d_model), dtype=np.float32)
+                           * np.float32(1.0 / np.sqrt(d_model)))
+    return x, w
 
 
 def make_inputs(w: Workload, seed: int, cache_capacity: Optional[int] = None) -> Dict[str, np.ndarray]:

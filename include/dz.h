@@ -108,6 +108,12 @@ typedef enum {
   DZ_MODE_CROSS = 3
 } dz_mode;
 
+/* Flag OR-ed into dz_chunk_layout.mode: q and the call's own k are already
+ * rotated (for example by dz_qkv_rope), so the call does not rotate them.
+ * Cache keys are always used as stored.  An interface choice of this library;
+ * the pages have no counterpart. */
+#define DZ_MODE_ROTATED 0x100
+
 /* Token layout of one call.  A chunk is frames_per_chunk latent frames of
  * grid_h x grid_w tokens, frame-major then row then column, followed by
  * n_action action tokens: chunk_len L = F*grid_h*grid_w + n_action.
@@ -205,6 +211,30 @@ dz_status dz_kvcache_append(dz_attn_t handle, dz_kvcache* cache, const void* k, 
  * DZ_ERR_ALIGNMENT, DZ_ERR_CUDA. */
 dz_status dz_kvcache_replace(dz_attn_t handle, dz_kvcache* cache, int32_t chunk_index,
                              const void* k, const void* v, void* stream);
+
+/* QKV projection with the rotary embedding and the KV-cache append fused into
+ * one GEMM ("DreamZero (WAM) 模型架构", §2.3 block diagram: the causal
+ * self-attention of each DiT block takes the normalised, modulated hidden
+ * state [B, T, 5120]; RoPE acts on the latent sequence).  For the S tokens of
+ * each batch item:
+ *   [q | k | v] = x W^T  (fp32 accumulation of bf16 products),
+ *   q, k turned by R(pos(s)) in fp32 (the rule of dz_rope3d: token s is token
+ *   s % L of chunk first_chunk + s / L of `layout`), then q, k, v rounded once
+ *   to bf16.
+ *   x    bf16 [B][S][d_model], row-major; d_model a positive multiple of 64.
+ *   w    bf16 [3 * H * 128][d_model]: row n is output feature n; rows
+ *        [0, H*128) give q (head-major, 128 per head), then k, then v.
+ *   q_out, k_out, v_out  bf16 [B][S][H][128] (H = the handle's num_heads).
+ *   cache  NULL, or a cache to append to: k and v are also written to rows
+ *        [len_tokens, len_tokens + S) of every batch item and len_tokens
+ *        advances by S (S must equal cache->chunk_len; batch must match).
+ * No bias term (the pages give none).  All pointers 16-byte aligned.
+ * Errors: DZ_ERR_INVALID_ARG, DZ_ERR_ALIGNMENT, DZ_ERR_SHAPE (d_model, or
+ * positions beyond the handle's tables), DZ_ERR_CAPACITY (batch beyond the
+ * handle, cache full), DZ_ERR_CUDA; nothing is written on error. */
+dz_status dz_qkv_rope(dz_attn_t handle, const void* x, const void* w, int32_t B, int32_t S,
+                      int32_t d_model, const dz_chunk_layout* layout, int32_t first_chunk,
+                      void* q_out, void* k_out, void* v_out, dz_kvcache* cache, void* stream);
 
 /* The same attention as dz_chunk_attn_forward, for callers that cannot call
  * cudaMalloc: code that runs while a stream is being captured in global mode,

@@ -160,6 +160,32 @@ def rope3d(x: np.ndarray, F: int, gh: int, gw: int, n_action: int, t_offset: int
     return rotate_pairs(x, rope_angles(t, h, w, spec))
 
 
+def qkv_rope(x_bits: np.ndarray, w_bits: np.ndarray, heads: int, F: int, gh: int, gw: int,
+             n_action: int, t_offset: int, first_chunk: int, spec: RopeSpec = RopeSpec()):
+    """dz_qkv_rope: the attention inputs of a run of chunk tokens.
+
+    The causal self-attention of a DiT block projects the block's hidden state
+    [B, T, 5120] to q, k, v ("DreamZero (WAM) 模型架构", §2.3 block diagram) and
+    RoPE acts on the latent sequence.  Here [q | k | v] = x W^T (no bias: the
+    pages give none) from the exact bf16 values in float64, split into heads of
+    128 features (feature n of a section belongs to head n // 128), then q and k
+    are rotated at their tokens' positions by ``rope3d``.  Returns float64
+    q, k, v, each [B, S, heads, 128].
+    """
+    x = widen_bf16(x_bits)                 # [B, S, d_model]
+    w = widen_bf16(w_bits)                 # [3 * heads * D, d_model]
+    D = spec.head_dim
+    B, S = x.shape[0], x.shape[1]
+    y = x @ w.T                            # [B, S, 3 * heads * D]
+    HD = heads * D
+    q = y[..., :HD].reshape(B, S, heads, D)
+    k = y[..., HD:2 * HD].reshape(B, S, heads, D)
+    v = y[..., 2 * HD:].reshape(B, S, heads, D)
+    q = rope3d(q, F, gh, gw, n_action, t_offset, first_chunk, spec)
+    k = rope3d(k, F, gh, gw, n_action, t_offset, first_chunk, spec)
+    return q, k, v
+
+
 # ---------------------------------------------------------------------------
 # Visibility (the chunk mask)
 # ---------------------------------------------------------------------------

@@ -419,3 +419,46 @@ def test_workload4_long_cache_and_cross():
     gx = run_forward(xl, w.heads, inp["q_x"], inp["k_x"], inp["v_x"])
     rx = oracle_full(xl, inp["q_x"], inp["k_x"], inp["v_x"])
     assert_close(gx, rx, w.name + " cross")
+
+
+def test_workload5_three_view_grid_decode():
+    """Three camera views tiled into one 22x40 latent grid (880 tokens per frame)."""
+    w = WORKLOADS[5]
+    inp = synth.make_inputs(w, 5)
+    got = run_forward(w.layout, w.heads, inp["q"], inp["k"], inp["v"], inp["cache_k"],
+                      inp["cache_v"], w.cache_tokens)
+    ref = oracle_full(w.layout, inp["q"], inp["k"], inp["v"], inp["cache_k"], inp["cache_v"],
+                      w.cache_tokens)
+    assert_close(got, ref, w.name)
+
+
+def test_window_reset_restarts_positions():
+    """At a local-attention window boundary the old keys and values are dropped and
+    frame positions restart at zero: after len_tokens = 0 and t_offset = 0, appending
+    chunk A (rotated at chunk 0) and decoding chunk B gives the rows of a fresh
+    two-chunk block-causal prefill, whatever the old window left in the buffer."""
+    rng = np.random.default_rng(33)
+    F, gh, gw, na, H = 1, 8, 8, 8, 2
+    L = F * gh * gw + na
+    h = handle(H)
+    cap = 4 * L
+    ck = to_dev(rand_bits(rng, (1, cap, H, D), 2.0))   # the old window's contents
+    cv = to_dev(rand_bits(rng, (1, cap, H, D), 2.0))
+    cache = dz.make_cache(ck, cv, 1, cap, 3 * L, L)
+    # reset at the window boundary
+    cache.len_tokens = 0
+    q = rand_bits(rng, (1, 2 * L, H, D))
+    k = rand_bits(rng, (1, 2 * L, H, D))
+    v = rand_bits(rng, (1, 2 * L, H, D))
+    ka = to_dev(k[:, :L])
+    ka_rot = torch.empty_like(ka)
+    dz.dz_rope3d(h, ka, ka_rot, 1, L, dz.make_layout(MODE_PREFILL, 1, F, gh, gw, na, 1), 0)
+    dz.dz_kvcache_append(h, cache, ka_rot, to_dev(v[:, :L]))
+    assert cache.len_tokens == L
+    out = torch.empty((1, L, H, D), dtype=torch.bfloat16, device="cuda")
+    dz.dz_chunk_attn_forward(h, to_dev(q[:, L:]), to_dev(k[:, L:]), to_dev(v[:, L:]), cache,
+                             dz.make_layout(MODE_DECODE, 1, F, gh, gw, na, 1, 0), out)
+    dz.dz_attn_sync_status(h)
+    lay_p = L_(MODE_PREFILL, 1, F, gh, gw, na, 2)
+    ref = oracle_full(lay_p, q, k, v)[:, L:]
+    assert_close(to_f64(out), ref, "decode after window reset")

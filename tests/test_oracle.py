@@ -307,10 +307,50 @@ def pin_decode_equals_prefill():
     np.testing.assert_allclose(dec, full[:, n * L:], rtol=0, atol=1e-13)
 
 
+def pin_qkv_identity_blocks():
+    """With W = [I; 2I; -I] (d_model = H*128) the projection copies x: q is x rotated,
+    k is 2x rotated, v is -x unrotated; fixes the q/k/v section order, the head
+    layout of the features and which sections turn."""
+    rng = np.random.default_rng(41)
+    H, F, gh, gw, na = 2, 1, 2, 3, 2
+    L = O.chunk_len(F, gh, gw, na)
+    S = 2 * L
+    x = _rand_bits(rng, (1, S, H * D))
+    eye = np.eye(H * D)
+    w = _bits(np.concatenate([eye, 2 * eye, -eye]))
+    q, k, v = O.qkv_rope(x, w, H, F, gh, gw, na, 5, 1)
+    xs = O.widen_bf16(x).reshape(1, S, H, D)
+    for s in range(S):
+        pos = bf._grid_pos(s % L, 1 + s // L, F, gh, gw, 5)
+        for h in range(H):
+            ref = bf.rotate_token(xs[0, s, h].tolist(), pos)
+            np.testing.assert_allclose(q[0, s, h], ref, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(k[0, s, h], 2 * np.array(ref), rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(v, -xs)
+
+
+def pin_qkv_brute_force():
+    """One token's q, k, v by explicit sums over d_model and the complex-number
+    rotation, against the oracle's matmul + 2x2 rotation."""
+    rng = np.random.default_rng(42)
+    H, dm, F, gh, gw, na = 1, 64, 2, 2, 2, 1
+    L = O.chunk_len(F, gh, gw, na)
+    x = _rand_bits(rng, (1, L, dm))
+    w = _rand_bits(rng, (3 * H * D, dm), 0.2)
+    q, k, v = O.qkv_rope(x, w, H, F, gh, gw, na, 0, 2)
+    xf, wf = O.widen_bf16(x), O.widen_bf16(w)
+    for s in (0, 5, L - 1):
+        y = [math.fsum(xf[0, s, c] * wf[n, c] for c in range(dm)) for n in range(3 * D)]
+        pos = bf._grid_pos(s, 2, F, gh, gw, 0)
+        np.testing.assert_allclose(q[0, s, 0], bf.rotate_token(y[:D], pos), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(k[0, s, 0], bf.rotate_token(y[D:2 * D], pos), rtol=0, atol=1e-11)
+        np.testing.assert_allclose(v[0, s, 0], y[2 * D:], rtol=0, atol=1e-11)
+
+
 ALL_PINS = [pin_visibility_golden, pin_positions_golden, pin_attention_closed_forms,
             pin_rope_invariants, pin_rope_relative, pin_brute_force, pin_library_sdpa,
             pin_softmax_rows, pin_single_visible_key, pin_equal_scores, pin_causality,
-            pin_decode_equals_prefill]
+            pin_decode_equals_prefill, pin_qkv_identity_blocks, pin_qkv_brute_force]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
@@ -456,7 +496,24 @@ def _row_major_frames(n_tokens, F, gh, gw, n_action, t_offset, first_chunk):
     return t, w % gh if gh > 1 else h, h % gw if gw > 1 else w
 
 
+_orig_qkv = O.qkv_rope
+
+
+def _qkv_rotates_v(x_bits, w_bits, heads, F, gh, gw, n_action, t_offset, first_chunk,
+                   spec=O.RopeSpec()):
+    q, k, v = _orig_qkv(x_bits, w_bits, heads, F, gh, gw, n_action, t_offset, first_chunk, spec)
+    return q, k, O.rope3d(v, F, gh, gw, n_action, t_offset, first_chunk, spec)
+
+
+def _qkv_sections_swapped(x_bits, w_bits, heads, F, gh, gw, n_action, t_offset, first_chunk,
+                          spec=O.RopeSpec()):
+    q, k, v = _orig_qkv(x_bits, w_bits, heads, F, gh, gw, n_action, t_offset, first_chunk, spec)
+    return k, q, v
+
+
 PLANTED = [
+    ("qkv_rope", _qkv_rotates_v),
+    ("qkv_rope", _qkv_sections_swapped),
     ("rotate_pairs", _wrong_sign_rotate),
     ("rope_angles", _swapped_axes_angles),
     ("rope_angles", _split_21_22_21),
