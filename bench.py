@@ -240,6 +240,73 @@ def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float)
     return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
+def e2e_pipelined(dev, stream, dev_inputs: dict, dev_outputs: dict, call, n_steps: int,
+                  world: int) -> dict:
+    """End-to-end steps through the public calls: every step copies its inputs in from
+    pinned host memory and its results back out.  Two slots: while step i runs on
+    `stream`, the inputs of step i+1 and the results of step i-1 cross PCIe on their
+    own streams (event-ordered).  Returns ms for n_steps (max over ranks) and bytes."""
+    import torch
+    host_in = {k: t.cpu().pin_memory() for k, t in dev_inputs.items()}
+    host_out = [{k: torch.empty_like(t, device="cpu").pin_memory() for k, t in dev_outputs.items()}
+                for _ in range(2)]
+    dev_in = [{k: torch.empty_like(t) for k, t in dev_inputs.items()} for _ in range(2)]
+    dev_out = [{k: torch.empty_like(t) for k, t in dev_outputs.items()} for _ in range(2)]
+    h2d_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]    # inputs of the slot landed
+    ev_comp = [torch.cuda.Event() for _ in range(2)]  # the call is done with the slot
+    ev_out = [torch.cuda.Event() for _ in range(2)]   # the slot's results are on the host
+    step_no = [0]
+
+    def step():
+        i = step_no[0]
+        sl = i % 2
+        step_no[0] += 1
+        if i >= 2:
+            h2d_stream.wait_event(ev_comp[sl])
+        with torch.cuda.stream(h2d_stream):
+            for k in host_in:
+                dev_in[sl][k].copy_(host_in[k], non_blocking=True)
+            ev_in[sl].record(h2d_stream)
+        stream.wait_event(ev_in[sl])
+        if i >= 2:
+            stream.wait_event(ev_out[sl])
+        call(dev_in[sl], dev_out[sl])
+        ev_comp[sl].record(stream)
+        d2h_stream.wait_event(ev_comp[sl])
+        with torch.cuda.stream(d2h_stream):
+            for k in host_out[sl]:
+                host_out[sl][k].copy_(dev_out[sl][k], non_blocking=True)
+            ev_out[sl].record(d2h_stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    x0 = torch.cuda.Event(enable_timing=True)
+    x1 = torch.cuda.Event(enable_timing=True)
+    x0.record(h2d_stream)
+    stream.wait_event(x0)
+    d2h_stream.wait_event(x0)
+    for _ in range(n_steps):
+        step()
+    stream.wait_event(ev_out[(step_no[0] - 1) % 2])
+    stream.wait_event(ev_out[step_no[0] % 2])
+    x1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(x0.elapsed_time(x1), world, dev)
+    return {"unit": "TFLOP/s", "ms": ms, "steps_done": n_steps,
+            "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in host_in.values())),
+            "d2h_bytes_per_step": int(sum(t.numel() * t.element_size()
+                                          for t in host_out[0].values())),
+            "pipelined": "inputs of step i+1 and the results of step i-1 cross PCIe while "
+                         "step i runs",
+            "ms_per_step": round(ms / n_steps, 4), "steps": n_steps}
+
+
 # ----------------------------------------------------------------------------------- GPU leg
 
 def run_gpu(args, rank: int, world: int, local_rank: int):
@@ -344,78 +411,150 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     s0 = sets[0]
     in_keys = [k for k in ("q", "k", "v", "q_x", "k_x", "v_x") if k in s0]
     out_keys = [k for k in ("out", "out_x") if k in s0]
-    host_in = {k: s0[k].cpu().pin_memory() for k in in_keys}
-    # two slots: while step i computes, step i+1's inputs are copied in and step
-    # i-1's result is copied out (separate copy streams, event-ordered)
-    host_out = [{k: torch.empty_like(s0[k], device="cpu").pin_memory() for k in out_keys}
-                for _ in range(2)]
-    dev_in = [{k: torch.empty_like(s0[k]) for k in in_keys} for _ in range(2)]
-    dev_out = [{k: torch.empty_like(s0[k]) for k in out_keys} for _ in range(2)]
-    h2d_stream = torch.cuda.Stream(device=dev)
-    d2h_stream = torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]      # inputs of the slot landed
-    ev_used = [torch.cuda.Event() for _ in range(2)]    # the call has read the slot's inputs
-    ev_comp = [torch.cuda.Event() for _ in range(2)]    # the slot's result is written
-    ev_out = [torch.cuda.Event() for _ in range(2)]     # the slot's result is on the host
-    n_e2e = max(3, min(args.steps, 200))
-    step_no = [0]
 
-    def e2e_step():
-        i = step_no[0]
-        sl = i % 2
-        step_no[0] += 1
-        if i >= 2:
-            h2d_stream.wait_event(ev_used[sl])
-        with torch.cuda.stream(h2d_stream):
-            for k in in_keys:
-                dev_in[sl][k].copy_(host_in[k], non_blocking=True)
-            ev_in[sl].record(h2d_stream)
-        stream.wait_event(ev_in[sl])
-        if i >= 2:
-            stream.wait_event(ev_out[sl])
-        di, do = dev_in[sl], dev_out[sl]
+    def e2e_call(di, do):
         dz.dz_chunk_attn_forward(h, di["q"], di["k"], di["v"], s0["cache"], dl, do["out"], stream)
         if dlx is not None:
             dz.dz_chunk_attn_forward(h, di["q_x"], di["k_x"], di["v_x"], None, dlx,
                                      do["out_x"], stream)
-        ev_used[sl].record(stream)
-        ev_comp[sl].record(stream)
-        d2h_stream.wait_event(ev_comp[sl])
-        with torch.cuda.stream(d2h_stream):
-            for k in out_keys:
-                host_out[sl][k].copy_(do[k], non_blocking=True)
-            ev_out[sl].record(d2h_stream)
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    x0 = torch.cuda.Event(enable_timing=True)
-    x1 = torch.cuda.Event(enable_timing=True)
-    x0.record(h2d_stream)
-    stream.wait_event(x0)
-    d2h_stream.wait_event(x0)
-    for _ in range(n_e2e):
-        e2e_step()
-    stream.wait_event(ev_out[(step_no[0] - 1) % 2])
-    stream.wait_event(ev_out[step_no[0] % 2])
-    x1.record(stream)
-    torch.cuda.synchronize(dev)
-    ems = x0.elapsed_time(x1)
-    ems = max_over_ranks(ems, world, dev)
+    e2e = e2e_pipelined(dev, stream, {k: s0[k] for k in in_keys}, {k: s0[k] for k in out_keys},
+                        e2e_call, max(3, min(args.steps, 200)), world)
     dz.dz_attn_sync_status(h, stream)
-    e2e = {"value": round(job_throughput(flops, n_e2e, world, ems), 3), "unit": "TFLOP/s",
-           "h2d_bytes_per_step": int(sum(host_in[k].numel() * 2 for k in in_keys)),
-           "d2h_bytes_per_step": int(sum(host_out[0][k].numel() * 2 for k in out_keys)),
-           "pipelined": "inputs of step i+1 and the result of step i-1 cross PCIe while step i runs",
-           "ms_per_step": round(ems / n_e2e, 4), "steps": n_e2e}
+    e2e["value"] = round(job_throughput(flops, e2e.pop("steps_done"), world, e2e.pop("ms")), 3)
 
     for gr in graphs.values():
         del gr
     graphs.clear()
     dz.dz_attn_destroy(h)
     return ms_per_step, tflops_total, clocks, e2e
+
+
+QKV_METRIC = ("fused QKV projection + 3D RoPE TFLOP/s and % of B200 BF16 peak; "
+              "\u00b5s per DiT-layer projection of one chunk")
+D_MODEL = 5120  # hidden size of the 14B DiT
+
+
+def qkv_flops(w) -> float:
+    lay = w.layout
+    return 2.0 * lay.batch * lay.chunk_len * D_MODEL * 3 * w.heads * w.head_dim
+
+
+def time_graph(stream, call, steps: int, warmup: int, world: int, dev, sampler=None):
+    """Device time (ms, max over ranks) of `steps` calls replayed from CUDA graphs of up to
+    240 calls, after `warmup` plain calls and one replay of each graph."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            call(i)
+    stream.synchronize()
+    g = min(240, steps)
+    full, rem = divmod(steps, g)
+    graphs = {}
+    for n in ([g] if full else []) + ([rem] if rem else []):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for i in range(n):
+                call(i)
+        graphs[n] = gr
+    with torch.cuda.stream(stream):
+        for gr in graphs.values():
+            gr.replay()
+    stream.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(full):
+            graphs[g].replay()
+        if rem:
+            graphs[rem].replay()
+        e1.record(stream)
+    stream.synchronize()
+    clocks = sampler.stop() if sampler else None
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    graphs.clear()
+    return ms, clocks
+
+
+def run_qkv(args, rank: int, world: int, local_rank: int, config: dict):
+    """Times dz_qkv_rope on one chunk of the workload (d_model 5120, random weights)."""
+    import torch
+    from causal_video_diffusion_rope_b200 import dz
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    lay = w.layout
+    B, H, D, S = lay.batch, w.heads, w.head_dim, lay.chunk_len
+    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B))
+    dl = dz.layout_from(lay)
+    first = lay.num_chunks if lay.mode == synth.MODE_DECODE else 0
+    xs, W = [], None
+    for i in range(2):
+        xb, wb = synth.projection_inputs(1000 * rank + i, B, S, D_MODEL, H)
+        xs.append(torch.from_numpy(xb.view(np.int16)).to(dev).view(torch.bfloat16))
+        if W is None:
+            W = torch.from_numpy(wb.view(np.int16)).to(dev).view(torch.bfloat16)
+    q = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
+    k, v = torch.empty_like(q), torch.empty_like(q)
+    stream = torch.cuda.Stream(device=dev)
+
+    def call(i):
+        dz.dz_qkv_rope(h, xs[i % 2], W, B, S, D_MODEL, dl, first, q, k, v, None, stream)
+
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    ms, clocks = time_graph(stream, call, args.steps, args.warmup, world, dev, sampler)
+    dz.dz_attn_sync_status(h, stream)
+    ms_per_step = ms / args.steps
+    flops = qkv_flops(w)
+
+    # context: cuBLAS (torch.matmul) on the same GEMM alone, no rotation, same timing
+    x2 = [x.view(B * S, D_MODEL) for x in xs]
+    y = torch.empty((B * S, 3 * H * D), dtype=torch.bfloat16, device=dev)
+
+    def call_ref(i):
+        torch.matmul(x2[i % 2], W.t(), out=y)
+
+    ms_ref, _ = time_graph(stream, call_ref, min(args.steps, 2400), 3, world, dev)
+    ref_us = 1e3 * ms_ref / min(args.steps, 2400)
+
+    def e2e_call(di, do):
+        dz.dz_qkv_rope(h, di["x"], W, B, S, D_MODEL, dl, first, do["q"], do["k"], do["v"],
+                       None, stream)
+
+    e2e = e2e_pipelined(dev, stream, {"x": xs[0]}, {"q": q, "k": k, "v": v}, e2e_call,
+                        max(3, min(args.steps, 200)), world)
+    e2e["value"] = round(job_throughput(flops, e2e.pop("steps_done"), world, e2e.pop("ms")), 3)
+    dz.dz_attn_sync_status(h, stream)
+    dz.dz_attn_destroy(h)
+    if rank != 0:
+        return
+    peak_tf, _, peak_kind = measured_peaks()
+    per_gpu = flops / (ms_per_step * 1e-3) / 1e12
+    line = {"metric": QKV_METRIC, "value": round(job_throughput(flops, args.steps, world, ms), 3),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6), "us_per_call": round(ms_per_step * 1e3, 3),
+            "pct_of_bf16_peak": round(100 * per_gpu / peak_tf, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (x ~ N(0,1), random-init W ~ N(0, 1/5120))",
+            "config": dict(config, op="qkv_rope", d_model=D_MODEL, tokens=B * S,
+                           out_features=3 * H * D, flop_per_step=flops,
+                           l2="the 157 MB weight alone exceeds the 126 MB L2",
+                           parallelism=f"dp{world} (independent replicas of the call)"),
+            "roofline": {"bound": "tensor", "achieved": round(per_gpu, 2), "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": round(per_gpu / peak_tf, 4), "traffic": None,
+                         "peak_kind": f"{peak_kind} bf16 (burst)", "kernel": "qkv_rope_kernel"},
+            "context": {"cublas_same_gemm_us": round(ref_us, 3),
+                        "cublas_same_gemm_tflops": round(flops / (ref_us * 1e-6) / 1e12, 2)},
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
 
 
 def main():
@@ -426,6 +565,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle CPU work for the cpu_baseline field")
+    ap.add_argument("--op", default="attn", choices=["attn", "qkv"],
+                    help="attn: the chunk-causal attention call; qkv: the fused projection")
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
                     choices=range(len(synth.WORKLOADS)),
                     help="workload index (default: the single-layer inference step)")
@@ -444,6 +585,22 @@ def main():
               "cross_keys": w.cross_kv_len,
               "rope": "3d t/h/w 22/21/21 base 1e4; q and the chunk's k rotated once per call",
               "flop_per_step": step_flops(w)}
+
+    if args.op == "qkv":
+        if args.impl == "reference":
+            if rank == 0:
+                print(json.dumps({"impl": "reference", "unavailable": "the reference arm times "
+                                  "the attention call (--op attn) only"}), flush=True)
+            return
+        import torch.distributed as dist
+        if world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        run_qkv(args, rank, world, local_rank, config)
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
 
     if args.impl == "reference":
         if rank != 0:

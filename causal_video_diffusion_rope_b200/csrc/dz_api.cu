@@ -461,7 +461,7 @@ dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int3
     p.cache_cap = cache->capacity_tokens;
     p.cache_row0 = cache->len_tokens;
   }
-  // x as [M][d_model] with 64 x 128 boxes, w as [N][d_model] with 64 x 256 boxes
+  // x as [M][d_model] and w as [N][d_model], both with 64 x 256 boxes
   auto map2d = [&](CUtensorMap* m, const void* base, long long rows, int box_rows) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d_model) * 2};
@@ -473,7 +473,7 @@ dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int3
                                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? DZ_OK : DZ_ERR_CUDA;
   };
-  st = map2d(&p.tm_x, x, M, 128);
+  st = map2d(&p.tm_x, x, M, 256);
   if (st == DZ_OK) st = map2d(&p.tm_w, w, N, 256);
   if (st != DZ_OK) return st;
   p.q = q_out;

@@ -184,7 +184,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
 
 // Fused QKV projection + rotation (+ cache append); see dz_qkv.cu.
 struct QkvLaunch {
-  CUtensorMap tm_x, tm_w;  // x [M][K], w [3*H*128][K], bf16, 64 x (128 | 256) boxes, SW128
+  CUtensorMap tm_x, tm_w;  // x [M][K], w [3*H*128][K], bf16, 64 x 256 boxes, SW128
   void *q, *k, *v;         // [M][H][128]
   void *ck, *cv;           // cache or null
   int cache_cap, cache_row0;

@@ -11,13 +11,15 @@
 // ("DreamZero (WAM) 模型架构", §2.3 block diagram: RMSNorm, modulation, causal
 // self-attention with RoPE on the latent sequence).
 //
-// One persistent CTA per SM walks output tiles of 128 tokens x 256 features
+// One persistent CTA per SM walks output tiles of 256 tokens x 256 features
 // (two heads), n-tile major so that the CTAs working at one time share the
-// same weight tile through L2.  Warp 0 issues TMA loads of 64-wide K slices
-// into a 4-stage ring, warp 1 allocates TMEM and issues tcgen05.mma (M=128,
-// N=256, K=16, both operands K-major SW128 in shared memory), accumulating in
-// one of two 256-column TMEM buffers, and warps 2-5 drain the other buffer
-// (rotation, bf16 rounding, stores) while the next tile accumulates.
+// same weight tile through L2.  A tile is two 128-row halves that share each
+// weight slice, so every byte brought to the SM feeds twice the products of a
+// 128 x 256 tile.  Warp 0 issues TMA loads of 64-wide K slices into a 3-stage
+// ring, warp 1 allocates TMEM and issues tcgen05.mma (M=128, N=256, K=16, both
+// operands K-major SW128 in shared memory; two per K step, one per half) into
+// two 256-column TMEM accumulators, and warps 2-9 (one per TMEM lane quarter
+// and half) drain them (rotation, bf16 rounding, stores).
 #include "dz_internal.cuh"
 #include "dz_ptx.cuh"
 
@@ -25,9 +27,10 @@ namespace dz {
 
 namespace {
 
-constexpr int QBM = 128, QBN = 256, QBK = 64, QSTAGES = 4;
-constexpr int QTHREADS = 192;
-constexpr int QA_BYTES = QBM * QBK * 2;  // 16 KiB
+constexpr int QBM = 256, QBN = 256, QBK = 64, QSTAGES = 3;
+constexpr int QHALF = 128;               // rows per MMA (one TMEM lane each)
+constexpr int QTHREADS = 320;            // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int QA_BYTES = QBM * QBK * 2;  // 32 KiB
 constexpr int QB_BYTES = QBN * QBK * 2;  // 32 KiB
 constexpr int QSTAGE_BYTES = QA_BYTES + QB_BYTES;
 constexpr int QSM_BAR = QSTAGES * QSTAGE_BYTES;
@@ -39,8 +42,8 @@ enum {
   QB_FULL = 0,
   QB_EMPTY = QB_FULL + QSTAGES,
   QB_ACC_FULL = QB_EMPTY + QSTAGES,
-  QB_ACC_EMPTY = QB_ACC_FULL + 2,
-  QB_DRAIN = QB_ACC_EMPTY + 2,
+  QB_ACC_EMPTY = QB_ACC_FULL + 1,
+  QB_DRAIN = QB_ACC_EMPTY + 1,
   QB_COUNT = QB_DRAIN + 1
 };
 static_assert(QB_COUNT * 8 <= 256, "barrier area");
@@ -91,10 +94,8 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
       mbar_init(&bar[QB_FULL + s], 1);
       mbar_init(&bar[QB_EMPTY + s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bar[QB_ACC_FULL + b], 1);
-      mbar_init(&bar[QB_ACC_EMPTY + b], 128);
-    }
+    mbar_init(&bar[QB_ACC_FULL], 1);
+    mbar_init(&bar[QB_ACC_EMPTY], 8 * 32);
     mbar_init(&bar[QB_DRAIN], 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -135,17 +136,15 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
   } else if (warp == 1) {
     // ---------------- tcgen05 issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(QBM, QBN, false);
+      const uint32_t idesc = idesc_bf16(QHALF, QBN, false);
       const uint32_t base_lo = desc_lo(smem_u32(smem), 16);
       uint32_t it = 0;
       int lt = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++lt) {
-        const int buf = lt & 1;
-        // the epilogue has drained this buffer (tile lt - 2)
-        if (!mbar_wait(&bar[QB_ACC_EMPTY + buf], ((lt >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        // the epilogue has drained the accumulators (tile lt - 1)
+        if (!mbar_wait(&bar[QB_ACC_EMPTY], (lt & 1) ^ 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t d = tmem + buf * QBN;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int st = it % QSTAGES;
           const uint32_t ph = (it / QSTAGES) & 1;
@@ -154,27 +153,32 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
           const uint32_t a0 = base_lo + ((st * QSTAGE_BYTES) >> 4);
           const uint32_t b0 = a0 + (QA_BYTES >> 4);
 #pragma unroll
-          for (int kk = 0; kk < QBK / 16; ++kk)
-            mma_ss(d, desc_join(a0 + ((kk * 32) >> 4)), desc_join(b0 + ((kk * 32) >> 4)), idesc,
-                   (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < QBK / 16; ++kk) {
+            const uint64_t bd = desc_join(b0 + ((kk * 32) >> 4));
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+              mma_ss(tmem + hf * QBN,
+                     desc_join(a0 + ((hf * QHALF * QBK * 2 + kk * 32) >> 4)), bd, idesc,
+                     (kb > 0 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(&bar[QB_EMPTY + st]);
         }
         if (!ok) break;
-        mma_commit(&bar[QB_ACC_FULL + buf]);
+        mma_commit(&bar[QB_ACC_FULL]);
       }
       mma_commit(&bar[QB_DRAIN]);
       drain(&bar[QB_DRAIN], 0);
     }
   } else {
-    // ---------------- epilogue: warps 2..5, one token row per thread ----------------
+    // ---------------- epilogue: warps 2..9, one token row per thread ----------------
     const int quarter = warp & 3;
-    const int r = 32 * quarter + lane;
+    const int half = (warp - 2) >> 2;
+    const int r = half * QHALF + 32 * quarter + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
     const int HD = p.H * HEAD_DIM;
     int lt = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
-      const int buf = lt & 1;
-      if (!mbar_wait(&bar[QB_ACC_FULL + buf], (lt >> 1) & 1, abort_flag, p.status)) break;
+      if (!mbar_wait(&bar[QB_ACC_FULL], lt & 1, abort_flag, p.status)) break;
       tc_fence_after();
       const int nt = tile / p.m_tiles, mt = tile - nt * p.m_tiles;
       const int m = mt * QBM + r;
@@ -183,44 +187,55 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
       const int s = valid ? m - bb * p.S : 0;
       int t = 0, hh = 0, w = 0;
       token_pos(p.geom, s, p.first_chunk, t, hh, w);
+      // 32-column pieces in the order (dims 0-31 of both heads, dims 32-63 of both, ...)
+      // so that each set of 16 (cos, sin) entries is read once for the two heads
 #pragma unroll 1
-      for (int c = 0; c < QBN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_addr + buf * QBN + c * 32, v);
-        tmem_wait_ld();
-        if (c == QBN / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(&bar[QB_ACC_EMPTY + buf]);
-        }
-        const int n = nt * QBN + c * 32;  // feature of column 0 of this piece
-        if (n >= p.N) continue;
-        const int sec = n / HD;  // 0 q, 1 k, 2 v
-        const int rem = n - sec * HD;
-        const int head = rem / HEAD_DIM, d0 = rem - head * HEAD_DIM;
-        uint32_t pk[16];
-        if (sec < 2) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 cs = __ldg(p.rope.tab + rope_index(p.rope, (d0 >> 1) + i, t, hh, w));
-            const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
-            const float y0 = __fmaf_rn(x0, cs.x, -__fmul_rn(x1, cs.y));
-            const float y1 = __fmaf_rn(x0, cs.y, __fmul_rn(x1, cs.x));
-            pk[i] = pack_bf16x2(y0, y1);
-          }
-        } else {
+      for (int dq = 0; dq < HEAD_DIM / 32; ++dq) {
+        float2 cs[16];
+        if (nt * QBN < 2 * HD) {  // the tile holds q or k features
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            cs[i] = __ldg(p.rope.tab + rope_index(p.rope, dq * 16 + i, t, hh, w));
         }
-        if (valid) {
-          __nv_bfloat16* dst = (sec == 0 ? p.q : (sec == 1 ? p.k : p.v)) +
-                               (static_cast<size_t>(m) * p.H + head) * HEAD_DIM + d0;
-          store_piece(dst, pk);
-          if (sec > 0 && p.ck) {
-            __nv_bfloat16* cdst = (sec == 1 ? p.ck : p.cv) +
-                                  ((static_cast<size_t>(bb) * p.cache_cap + p.cache_row0 + s) * p.H + head) *
-                                      HEAD_DIM + d0;
-            store_piece(cdst, pk);
+#pragma unroll 1
+        for (int hp = 0; hp < QBN / HEAD_DIM; ++hp) {
+          const int c = hp * (HEAD_DIM / 32) + dq;
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_addr + half * QBN + c * 32, v);
+          tmem_wait_ld();
+          if (dq == HEAD_DIM / 32 - 1 && hp == QBN / HEAD_DIM - 1) {
+            tc_fence_before();
+            mbar_arrive(&bar[QB_ACC_EMPTY]);
+          }
+          const int n = nt * QBN + c * 32;  // feature of column 0 of this piece
+          if (n >= p.N) continue;
+          const int sec = n / HD;  // 0 q, 1 k, 2 v
+          const int rem = n - sec * HD;
+          const int head = rem / HEAD_DIM, d0 = rem - head * HEAD_DIM;
+          uint32_t pk[16];
+          if (sec < 2) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
+              const float y0 = __fmaf_rn(x0, cs[i].x, -__fmul_rn(x1, cs[i].y));
+              const float y1 = __fmaf_rn(x0, cs[i].y, __fmul_rn(x1, cs[i].x));
+              pk[i] = pack_bf16x2(y0, y1);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          }
+          if (valid) {
+            __nv_bfloat16* dst = (sec == 0 ? p.q : (sec == 1 ? p.k : p.v)) +
+                                 (static_cast<size_t>(m) * p.H + head) * HEAD_DIM + d0;
+            store_piece(dst, pk);
+            if (sec > 0 && p.ck) {
+              __nv_bfloat16* cdst = (sec == 1 ? p.ck : p.cv) +
+                                    ((static_cast<size_t>(bb) * p.cache_cap + p.cache_row0 + s) * p.H +
+                                     head) * HEAD_DIM + d0;
+              store_piece(cdst, pk);
+            }
           }
         }
       }
