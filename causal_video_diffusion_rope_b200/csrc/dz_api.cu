@@ -486,6 +486,14 @@ dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int3
   p.rope = tables_of(a);
   p.geom = g;
   p.first_chunk = first_chunk;
+  p.stage_t0 = g.t_offset + first_chunk * g.F;
+  p.stage_nt = ((S - 1) / g.L + 1) * g.F;
+  p.stage_ok = (static_cast<long long>(p.stage_nt) * a->desc.rope_pairs_t +
+                    static_cast<long long>(g.gh) * a->desc.rope_pairs_h +
+                    static_cast<long long>(g.gw) * a->desc.rope_pairs_w <=
+                dz::QKV_ROPE_STAGE_MAX)
+                   ? 1
+                   : 0;
   p.status = a->status;
   p.num_sms = a->num_sms;
   st = cuda_status(dz::launch_qkv_rope(p, static_cast<cudaStream_t>(stream)), "qkv launch");

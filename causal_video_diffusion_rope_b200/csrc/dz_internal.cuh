@@ -192,9 +192,12 @@ struct QkvLaunch {
   RopeTables rope;
   ChunkGeom geom;
   int first_chunk;
+  int stage_ok, stage_t0, stage_nt;  // rotary rows staged in shared memory (see AttnLaunch)
   int* status;
   int num_sms;
 };
+// Capacity (float2 entries) of the projection kernel's shared-memory rotary table.
+constexpr int QKV_ROPE_STAGE_MAX = 4096;
 cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream);
 
 // Workspace (in floats) one partial-result slot needs: Q_TILES * TILE_M rows of

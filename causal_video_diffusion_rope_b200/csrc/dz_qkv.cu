@@ -35,7 +35,8 @@ constexpr int QB_BYTES = QBN * QBK * 2;  // 32 KiB
 constexpr int QSTAGE_BYTES = QA_BYTES + QB_BYTES;
 constexpr int QSM_BAR = QSTAGES * QSTAGE_BYTES;
 constexpr int QSM_MISC = QSM_BAR + 256;
-constexpr int QSMEM_BYTES = QSM_MISC + 64 + 1024;  // + alignment slack
+constexpr int QSM_ROPE = QSM_MISC + 64;             // staged rotary rows of the call
+constexpr int QSMEM_BYTES = QSM_ROPE + QKV_ROPE_STAGE_MAX * 8 + 1024;  // + alignment slack
 static_assert(QSMEM_BYTES <= 232448, "shared memory");
 
 enum {
@@ -58,6 +59,7 @@ struct __align__(64) QkvParams {
   RopeTables rope;
   ChunkGeom geom;
   int first_chunk;
+  int stage_ok, stage_t0, stage_nt;
   int* status;
 };
 
@@ -176,6 +178,23 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
     const int r = half * QHALF + 32 * quarter + lane;
     const uint32_t lane_addr = static_cast<uint32_t>(32 * quarter) << 16;
     const int HD = p.H * HEAD_DIM;
+    // the call's rotary rows (t in [stage_t0, stage_t0 + stage_nt), every h < gh and
+    // w < gw) go to shared memory while the first tile accumulates
+    RopeTables rope = p.rope;
+    if (p.stage_ok) {
+      float2* st_tab = reinterpret_cast<float2*>(smem + QSM_ROPE);
+      const int nt_ = p.stage_nt * p.rope.pt, nh = p.geom.gh * p.rope.ph, nw = p.geom.gw * p.rope.pw;
+      const float2* gt = p.rope.tab + p.rope.off_t + p.stage_t0 * p.rope.pt;
+      const float2* gh = p.rope.tab + p.rope.off_h;
+      const float2* gw = p.rope.tab + p.rope.off_w;
+      for (int i = tid - 64; i < nt_ + nh + nw; i += QTHREADS - 64)
+        st_tab[i] = i < nt_ ? gt[i] : (i < nt_ + nh ? gh[i - nt_] : gw[i - nt_ - nh]);
+      named_bar_sync(1, QTHREADS - 64);
+      rope.tab = st_tab;
+      rope.off_t = -p.stage_t0 * p.rope.pt;
+      rope.off_h = nt_;
+      rope.off_w = nt_ + nh;
+    }
     int lt = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
       if (!mbar_wait(&bar[QB_ACC_FULL], lt & 1, abort_flag, p.status)) break;
@@ -195,7 +214,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
         if (nt * QBN < 2 * HD) {  // the tile holds q or k features
 #pragma unroll
           for (int i = 0; i < 16; ++i)
-            cs[i] = __ldg(p.rope.tab + rope_index(p.rope, dq * 16 + i, t, hh, w));
+            cs[i] = rope.tab[rope_index(rope, dq * 16 + i, t, hh, w)];
         }
 #pragma unroll 1
         for (int hp = 0; hp < QBN / HEAD_DIM; ++hp) {
@@ -281,6 +300,9 @@ cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream) {
   p.rope = a.rope;
   p.geom = a.geom;
   p.first_chunk = a.first_chunk;
+  p.stage_ok = a.stage_ok;
+  p.stage_t0 = a.stage_t0;
+  p.stage_nt = a.stage_nt;
   p.status = a.status;
   const int total = p.m_tiles * p.n_tiles;
   const int grid = total < a.num_sms ? total : a.num_sms;
