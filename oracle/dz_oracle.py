@@ -315,6 +315,62 @@ def chunk_attn_forward(q_bits: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarra
     return masked_attention(q, k, v, vis)
 
 
+def chunk_attn_backward_f64(q: np.ndarray, k: np.ndarray, v: np.ndarray, do: np.ndarray,
+                            mode: int, F: int, gh: int, gw: int, n_action: int, num_chunks: int,
+                            t_offset: int = 0, spec: RopeSpec = RopeSpec()):
+    """Gradients of sum(dO * O) for the PREFILL / TEACHER_FORCING self-attention call,
+    with respect to its unrotated q, k and v (float64 [B, S, H, D] each).
+
+    The forward is O = softmax(qr kr^T / sqrt(D) over the visible pairs) v with
+    qr = R q and kr = R k, R the per-token 3D rotation (an orthogonal map: a 2x2
+    rotation per pair).  By the chain rule, with P the probabilities:
+        dv  = P^T dO,   dP = dO v^T,   dS = P * (dP - rowsum(P * dP)),
+        dqr = dS kr / sqrt(D),   dkr = dS^T qr / sqrt(D),
+        dq = R^T dqr,   dk = R^T dkr   (R^T turns each pair back by -theta).
+    Training form of the same chunk mask (hyper.ai summary, "方法": teacher
+    forcing; the walkthrough's training objective, Fig. 14).
+    """
+    if mode not in (PREFILL, TEACHER_FORCING):
+        raise ValueError("the backward covers PREFILL and TEACHER_FORCING")
+    B, S, H, D = q.shape
+    L = chunk_len(F, gh, gw, n_action)
+    if mode == PREFILL:
+        theta = rope_angles(*token_positions(S, F, gh, gw, n_action, t_offset, 0), spec)
+    else:
+        half = num_chunks * L
+        th = rope_angles(*token_positions(half, F, gh, gw, n_action, t_offset, 0), spec)
+        theta = np.concatenate([th, th], axis=0)
+    qr = rotate_pairs(q, theta)
+    kr = rotate_pairs(k, theta)
+    visible = visibility(mode, L, num_chunks)
+    scale = 1.0 / math.sqrt(D)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    for b in range(B):
+        for hh in range(H):
+            P = softmax_probs((qr[b, :, hh] @ kr[b, :, hh].T) * scale, visible)
+            g = do[b, :, hh]
+            dv[b, :, hh] = P.T @ g
+            dP = g @ v[b, :, hh].T
+            dS = P * (dP - (P * dP).sum(axis=1, keepdims=True))
+            dq[b, :, hh] = dS @ kr[b, :, hh] * scale
+            dk[b, :, hh] = dS.T @ qr[b, :, hh] * scale
+    dq = rotate_pairs(dq, -theta)
+    dk = rotate_pairs(dk, -theta)
+    return dq, dk, dv
+
+
+def chunk_attn_backward(q_bits, k_bits, v_bits, do_bits, mode: int, F: int, gh: int, gw: int,
+                        n_action: int, num_chunks: int, t_offset: int = 0,
+                        heads: Optional[slice] = None, spec: RopeSpec = RopeSpec()):
+    """``chunk_attn_backward_f64`` on bf16 bit arrays (optionally a slice of heads)."""
+    hs = slice(None) if heads is None else heads
+    return chunk_attn_backward_f64(widen_bf16(q_bits[:, :, hs]), widen_bf16(k_bits[:, :, hs]),
+                                   widen_bf16(v_bits[:, :, hs]), widen_bf16(do_bits[:, :, hs]),
+                                   mode, F, gh, gw, n_action, num_chunks, t_offset, spec)
+
+
 def attention_rows(q_bits, k_bits, v_bits, rows, mode: int, F: int, gh: int, gw: int,
                    n_action: int, num_chunks: int, t_offset: int = 0, kv_len: int = 0,
                    cache_k_bits=None, cache_v_bits=None, cache_len: int = 0,

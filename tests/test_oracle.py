@@ -347,10 +347,77 @@ def pin_qkv_brute_force():
         np.testing.assert_allclose(v[0, s, 0], y[2 * D:], rtol=0, atol=1e-11)
 
 
+def _forward_f64(q, k, v, mode, F, gh, gw, na, N, t0):
+    """The oracle's forward on float64 inputs (rotation + masked attention)."""
+    L = O.chunk_len(F, gh, gw, na)
+    if mode == O.PREFILL:
+        qr = O.rope3d(q, F, gh, gw, na, t0, 0)
+        kr = O.rope3d(k, F, gh, gw, na, t0, 0)
+    else:
+        h = N * L
+        qr = np.concatenate([O.rope3d(q[:, :h], F, gh, gw, na, t0, 0),
+                             O.rope3d(q[:, h:], F, gh, gw, na, t0, 0)], axis=1)
+        kr = np.concatenate([O.rope3d(k[:, :h], F, gh, gw, na, t0, 0),
+                             O.rope3d(k[:, h:], F, gh, gw, na, t0, 0)], axis=1)
+    return O.masked_attention(qr, kr, v, O.visibility(mode, L, N))
+
+
+def pin_backward_finite_differences():
+    """Central differences of sum(dO * O) against the backward, for elements of q, k
+    and v in clean and noisy chunks (teacher forcing) and in prefill."""
+    rng = np.random.default_rng(51)
+    F, gh, gw, na, N, t0 = 1, 2, 2, 1, 2, 3
+    L = O.chunk_len(F, gh, gw, na)
+    for mode, S in ((O.TEACHER_FORCING, 2 * N * L), (O.PREFILL, N * L)):
+        q, k, v, do = (rng.standard_normal((1, S, 1, D)) for _ in range(4))
+        dq, dk, dv = O.chunk_attn_backward_f64(q, k, v, do, mode, F, gh, gw, na, N, t0)
+        h = 1e-6
+        for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+            for (s, d) in ((0, 0), (L + 1, 37), (S - 1, 101), (S // 2, 64)):
+                xp, xm = x.copy(), x.copy()
+                xp[0, s, 0, d] += h
+                xm[0, s, 0, d] -= h
+                def f(xx):
+                    qq, kk, vv = (xx if name == "q" else q, xx if name == "k" else k,
+                                  xx if name == "v" else v)
+                    return float((_forward_f64(qq, kk, vv, mode, F, gh, gw, na, N, t0) * do).sum())
+                fd = (f(xp) - f(xm)) / (2 * h)
+                assert abs(fd - g[0, s, 0, d]) <= 1e-6 * (1 + abs(fd)), (mode, name, s, d, fd, g[0, s, 0, d])
+
+
+def pin_backward_autograd():
+    """torch float64 autograd through rotation, masked softmax and PV against the
+    closed-form backward (two heads, batch 2, teacher forcing)."""
+    rng = np.random.default_rng(52)
+    F, gh, gw, na, N, t0 = 1, 2, 3, 2, 2, 1
+    L = O.chunk_len(F, gh, gw, na)
+    S = 2 * N * L
+    q, k, v, do = (rng.standard_normal((2, S, 2, D)) for _ in range(4))
+    dq, dk, dv = O.chunk_attn_backward_f64(q, k, v, do, O.TEACHER_FORCING, F, gh, gw, na, N, t0)
+    th = O.rope_angles(*O.token_positions(N * L, F, gh, gw, na, t0, 0), O.RopeSpec())
+    theta = torch.from_numpy(np.concatenate([th, th], axis=0))
+    c, sn = torch.cos(theta)[None, :, None, :], torch.sin(theta)[None, :, None, :]
+    vis = torch.from_numpy(O.visibility(O.TEACHER_FORCING, L, N))
+    tq, tk, tv = (torch.from_numpy(a).requires_grad_() for a in (q, k, v))
+
+    def rot(x):
+        x0, x1 = x[..., 0::2], x[..., 1::2]
+        return torch.stack([x0 * c - x1 * sn, x0 * sn + x1 * c], dim=-1).flatten(-2)
+
+    qr, kr = rot(tq), rot(tk)
+    scores = torch.einsum("bshd,bthd->bhst", qr, kr) / math.sqrt(D)
+    p = torch.softmax(scores.masked_fill(~vis, float("-inf")), dim=-1)
+    out = torch.einsum("bhst,bthd->bshd", p, tv)
+    (out * torch.from_numpy(do)).sum().backward()
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-11)
+
+
 ALL_PINS = [pin_visibility_golden, pin_positions_golden, pin_attention_closed_forms,
             pin_rope_invariants, pin_rope_relative, pin_brute_force, pin_library_sdpa,
             pin_softmax_rows, pin_single_visible_key, pin_equal_scores, pin_causality,
-            pin_decode_equals_prefill, pin_qkv_identity_blocks, pin_qkv_brute_force]
+            pin_decode_equals_prefill, pin_qkv_identity_blocks, pin_qkv_brute_force,
+            pin_backward_finite_differences, pin_backward_autograd]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda f: f.__name__)
@@ -511,7 +578,50 @@ def _qkv_sections_swapped(x_bits, w_bits, heads, F, gh, gw, n_action, t_offset, 
     return k, q, v
 
 
+_orig_bwd = O.chunk_attn_backward_f64
+
+
+def _bwd_without_rowsum(q, k, v, do, mode, F, gh, gw, n_action, num_chunks, t_offset=0,
+                        spec=O.RopeSpec()):
+    # dS = P * dP (the rowsum(P * dP) term dropped): recompute everything by hand
+    L = O.chunk_len(F, gh, gw, n_action)
+    S = q.shape[1]
+    if mode == O.PREFILL:
+        theta = O.rope_angles(*O.token_positions(S, F, gh, gw, n_action, t_offset, 0), spec)
+    else:
+        th = O.rope_angles(*O.token_positions(num_chunks * L, F, gh, gw, n_action, t_offset, 0), spec)
+        theta = np.concatenate([th, th], axis=0)
+    qr, kr = O.rotate_pairs(q, theta), O.rotate_pairs(k, theta)
+    vis = O.visibility(mode, L, num_chunks)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    sc = 1.0 / math.sqrt(q.shape[-1])
+    for b in range(q.shape[0]):
+        for hh in range(q.shape[2]):
+            P = O.softmax_probs((qr[b, :, hh] @ kr[b, :, hh].T) * sc, vis)
+            dv[b, :, hh] = P.T @ do[b, :, hh]
+            dS = P * (do[b, :, hh] @ v[b, :, hh].T)
+            dq[b, :, hh] = dS @ kr[b, :, hh] * sc
+            dk[b, :, hh] = dS.T @ qr[b, :, hh] * sc
+    return O.rotate_pairs(dq, -theta), O.rotate_pairs(dk, -theta), dv
+
+
+def _bwd_rotates_forward(q, k, v, do, mode, F, gh, gw, n_action, num_chunks, t_offset=0,
+                         spec=O.RopeSpec()):
+    # the gradients turned by +theta twice more instead of back by -theta
+    dq, dk, dv = _orig_bwd(q, k, v, do, mode, F, gh, gw, n_action, num_chunks, t_offset, spec)
+    L = O.chunk_len(F, gh, gw, n_action)
+    S = q.shape[1]
+    if mode == O.PREFILL:
+        theta = O.rope_angles(*O.token_positions(S, F, gh, gw, n_action, t_offset, 0), spec)
+    else:
+        th = O.rope_angles(*O.token_positions(num_chunks * L, F, gh, gw, n_action, t_offset, 0), spec)
+        theta = np.concatenate([th, th], axis=0)
+    return O.rotate_pairs(dq, 2 * theta), O.rotate_pairs(dk, 2 * theta), dv
+
+
 PLANTED = [
+    ("chunk_attn_backward_f64", _bwd_without_rowsum),
+    ("chunk_attn_backward_f64", _bwd_rotates_forward),
     ("qkv_rope", _qkv_rotates_v),
     ("qkv_rope", _qkv_sections_swapped),
     ("rotate_pairs", _wrong_sign_rotate),
