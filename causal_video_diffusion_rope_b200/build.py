@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdz.so")
-SOURCES = ["dz_api.cu", "dz_kernels.cu", "dz_attn.cu", "dz_qkv.cu"]
+SOURCES = ["dz_api.cu", "dz_kernels.cu", "dz_attn.cu", "dz_qkv.cu", "dz_bwd.cu"]
 HEADERS = ["dz_internal.cuh", "dz_ptx.cuh"]
 
 

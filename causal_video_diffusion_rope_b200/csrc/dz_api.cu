@@ -251,9 +251,11 @@ dz_status dz_rope3d(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
                      "rope3d launch");
 }
 
-dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const void* v,
-                                const dz_kvcache* cache, const dz_chunk_layout* l, void* out,
-                                void* stream) {
+// The attention call; with lse != null (training form) it also writes each query
+// row's log2-domain softmax normaliser.
+static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const void* v,
+                              const dz_kvcache* cache, const dz_chunk_layout* l, void* out,
+                              float* lse, void* stream) {
   if (!a || !q || !k || !v || !l || !out) return DZ_ERR_INVALID_ARG;
   // inputs already rotated: the flag is taken off a local copy of the layout
   const bool given_rotated = (l->mode & DZ_MODE_ROTATED) != 0;
@@ -377,6 +379,7 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
     p.stage_ok = 0;
   }
   p.out = out;
+  p.lse = lse;
   p.ws = a->ws;
   p.counters = a->counters;
   p.status = a->status;
@@ -392,6 +395,22 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
   if (st != DZ_OK) return st;
   return cuda_status(dz::launch_attention(p, static_cast<cudaStream_t>(stream)),
                      "attention launch");
+}
+
+dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const void* v,
+                                const dz_kvcache* cache, const dz_chunk_layout* l, void* out,
+                                void* stream) {
+  return attn_forward(a, q, k, v, cache, l, out, nullptr, stream);
+}
+
+dz_status dz_chunk_attn_forward_lse(dz_attn_t a, const void* q, const void* k, const void* v,
+                                    const dz_chunk_layout* l, void* out, void* lse,
+                                    void* stream) {
+  if (!l || !lse) return DZ_ERR_INVALID_ARG;
+  const int mode = l->mode & ~DZ_MODE_ROTATED;
+  if (mode != DZ_MODE_PREFILL && mode != DZ_MODE_TEACHER_FORCING) return DZ_ERR_UNSUPPORTED;
+  if (!aligned16(lse)) return DZ_ERR_ALIGNMENT;
+  return attn_forward(a, q, k, v, nullptr, l, out, static_cast<float*>(lse), stream);
 }
 
 dz_status dz_kvcache_append(dz_attn_t a, dz_kvcache* c, const void* k, const void* v,
@@ -500,6 +519,62 @@ dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int3
   if (st != DZ_OK) return st;
   if (cache) cache->len_tokens += S;
   return DZ_OK;
+}
+
+dz_status dz_chunk_attn_backward(dz_attn_t a, const void* q, const void* k, const void* v,
+                                 const void* out, const void* dout, const void* lse,
+                                 const dz_chunk_layout* l, void* dq, void* dk, void* dv,
+                                 void* stream) {
+  if (!a || !q || !k || !v || !out || !dout || !lse || !l || !dq || !dk || !dv)
+    return DZ_ERR_INVALID_ARG;
+  if (l->mode != DZ_MODE_PREFILL && l->mode != DZ_MODE_TEACHER_FORCING) return DZ_ERR_UNSUPPORTED;
+  dz_status st = check_geom(l);
+  if (st != DZ_OK) return st;
+  if (l->num_chunks < 1) return DZ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(lse) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return DZ_ERR_ALIGNMENT;
+  if (l->batch > a->desc.max_batch) return DZ_ERR_CAPACITY;
+  const int H = a->desc.num_heads;
+  const dz::ChunkGeom g = geom_of(l);
+  const long long S = (l->mode == DZ_MODE_TEACHER_FORCING ? 2LL : 1LL) * g.L * l->num_chunks;
+  if (S > a->desc.max_q_tokens) return DZ_ERR_CAPACITY;
+  // the rotated q, k go to the handle's rotation workspace and D to its split workspace
+  if (!a->rot_ws || S > a->rot_tokens) return DZ_ERR_CAPACITY;
+  const size_t ws_floats = 2ull * a->num_sms * dz::PART_FLOATS;
+  if (static_cast<size_t>(l->batch) * H * S > ws_floats) return DZ_ERR_CAPACITY;
+  st = check_positions(a, g, 0, l->num_chunks - 1);
+  if (st != DZ_OK) return st;
+  const size_t elems = static_cast<size_t>(l->batch) * S * H * dz::HEAD_DIM;
+  __nv_bfloat16* qr = static_cast<__nv_bfloat16*>(a->rot_ws);
+  __nv_bfloat16* kr = qr + elems;
+  const int period = l->mode == DZ_MODE_TEACHER_FORCING ? g.L * l->num_chunks : 0;
+  st = cuda_status(dz::launch_rope3d(q, qr, l->batch, static_cast<int>(S), H, g, 0, tables_of(a),
+                                     static_cast<cudaStream_t>(stream), k, kr, period),
+                   "backward rotation launch");
+  if (st != DZ_OK) return st;
+  dz::BwdLaunch p;
+  st = make_map(a, &p.tm_q, qr, l->batch, static_cast<int>(S), static_cast<int>(S), H);
+  if (st == DZ_OK) st = make_map(a, &p.tm_k, kr, l->batch, static_cast<int>(S), static_cast<int>(S), H);
+  if (st == DZ_OK) st = make_map(a, &p.tm_v, v, l->batch, static_cast<int>(S), static_cast<int>(S), H);
+  if (st == DZ_OK) st = make_map(a, &p.tm_do, dout, l->batch, static_cast<int>(S), static_cast<int>(S), H);
+  if (st != DZ_OK) return st;
+  p.out = out;
+  p.dout = dout;
+  p.lse = static_cast<const float*>(lse);
+  p.dd = a->ws;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.rope = tables_of(a);
+  p.geom = g;
+  p.mode = l->mode;
+  p.N = l->num_chunks;
+  p.S = static_cast<int>(S);
+  p.B = l->batch;
+  p.H = H;
+  p.status = a->status;
+  return cuda_status(dz::launch_backward(p, static_cast<cudaStream_t>(stream)), "backward launch");
 }
 
 dz_status dz_attn_sync_status(dz_attn_t a, void* stream) {

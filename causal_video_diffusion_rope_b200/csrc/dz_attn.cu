@@ -94,6 +94,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory");
 struct __align__(64) AttnParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_ck, tm_cv;
   __nv_bfloat16* out;
+  float* lse;  // null, or log2-domain softmax normaliser per (b, h, query row)
   float* ws;
   int* counters;
   int* status;
@@ -791,6 +792,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // bf16 out = O / l; each 32-column chunk goes through the warp's transpose
         // buffer so that global stores cover 64 contiguous bytes of 8 rows at a time
         const float inv_l = 1.f / l_run;
+        if (p.lse && s_tok < p.sched.Sq)
+          p.lse[(static_cast<size_t>(b) * p.H + h) * p.sched.Sq + s_tok] = m_run + __log2f(l_run);
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
@@ -930,6 +933,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_wait_st();
           }
           const float invL = 1.f / Lsum;
+          if (p.lse && s_tok < p.sched.Sq)
+            p.lse[(static_cast<size_t>(b) * p.H + h) * p.sched.Sq + s_tok] = M + __log2f(Lsum);
 #pragma unroll 1
           for (int g = 0; g < 4; ++g) {  // 32 output columns per pass
             uint32_t v[32];
@@ -1001,6 +1006,7 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   p.tm_ck = a.tm_ck;
   p.tm_cv = a.tm_cv;
   p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.lse = a.lse;
   p.ws = a.ws;
   p.counters = a.counters;
   p.status = a.status;

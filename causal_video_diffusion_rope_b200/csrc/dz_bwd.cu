@@ -1,0 +1,630 @@
+// Backward of the prefill / teacher-forcing chunk-causal attention (training
+// form of the chunk mask: hyper.ai summary of the paper, "方法" (teacher
+// forcing); the walkthrough's training objective, Fig. 14).
+//
+// With qr = R q, kr = R k (per-token 3D rotation), S = qr kr^T / sqrt(128) over
+// the visible pairs, P = softmax(S) (from the forward's per-row log2 normaliser
+// lse), O = P v and the incoming dO:
+//   D = rowsum(dO * O),  dP = dO v^T,  dS = P * (dP - D),
+//   dv = P^T dO,  dqr = dS kr / sqrt(128),  dkr = dS^T qr / sqrt(128),
+//   dq = R^T dqr,  dk = R^T dkr.
+// Two kernels recompute S and dP instead of exchanging partial sums:
+//   bwd_dq_kernel   one CTA per (batch, head, 128-query tile): over the key tiles
+//                   it sees, S = Q K^T and dP = dO V^T (both operands K-major in
+//                   shared memory), dS in registers, written as bf16 over S in
+//                   TMEM, then dQ += dS K with dS read from TMEM;
+//   bwd_dkv_kernel  one CTA per (batch, head, 128-key tile): over the query tiles
+//                   that see it, S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
+//                   written as bf16 over them in TMEM, then dV += P^T dO and
+//                   dK += dS^T Q.
+// Each has a TMA warp (2-stage ring of the streamed tiles), an MMA warp and four
+// warps that own one TMEM lane (one tile row) per thread.  The rotation back
+// (R^T) and the 1/sqrt(128) are applied to the fp32 accumulators in the epilogue.
+#include "dz_internal.cuh"
+#include "dz_ptx.cuh"
+
+namespace dz {
+
+namespace {
+
+constexpr int BT = 128;                            // rows of a query or key tile
+constexpr int BTHREADS = 192;                      // warp 0 TMA, 1 MMA, 2-5 compute
+constexpr int BTILE = BT * HEAD_DIM * 2;           // 32 KiB
+constexpr int BHALF = BTILE / 2;                   // 64 dims x 128 rows
+constexpr int BSM_FIXED0 = 0;                      // resident tile 0 (Q or K)
+constexpr int BSM_FIXED1 = BTILE;                  // resident tile 1 (dO or V)
+constexpr int BSM_RING = 2 * BTILE;                // 2 stages x 2 tiles
+constexpr int BSM_BAR = BSM_RING + 4 * BTILE;
+constexpr int BSM_MISC = BSM_BAR + 256;
+constexpr int BSM_VEC = BSM_MISC + 64;             // lse and D of 128 queries, 2 buffers
+constexpr int BSMEM_BYTES = BSM_VEC + 2 * 2 * BT * 4 + 1024;
+static_assert(BSMEM_BYTES <= 232448, "shared memory");
+
+enum {
+  BB_FIX = 0,         // resident tiles landed
+  BB_FULL = 1,        // [2] ring stage landed
+  BB_EMPTY = 3,       // [2] ring stage consumed
+  BB_SDP = 5,         // S and dP (or their transposes) in TMEM
+  BB_READY = 6,       // compute warps wrote the bf16 operands (128 arrivals)
+  BB_ACC = 7,         // accumulators final
+  BB_DRAIN = 8,
+  BB_COUNT = 9
+};
+
+struct __align__(64) BwdParams {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // rotated q, rotated k, v, dO: (128, H, S, B)
+  const float* lse;                      // [B][H][S], log2 domain
+  const float* dd;                       // D = rowsum(dO * O), [B][H][S]
+  __nv_bfloat16 *dq, *dk, *dv;           // [B][S][H][128]
+  RopeTables rope;
+  ChunkGeom geom;
+  int mode, L, N, S;                     // S tokens per batch item (queries = keys)
+  int B, H, n_tiles;
+  int period;                            // TF: N*L (noisy tokens sit at clean positions)
+  float scale_log2, scale;
+  int* status;
+};
+
+// Visible keys of query s: [a0, a1) and [b0, b1).
+__device__ __forceinline__ void q_keys(const BwdParams& p, int s, int& a0, int& a1, int& b0,
+                                       int& b1) {
+  const int c = s / p.L;
+  a0 = 0;
+  b0 = b1 = 0;
+  if (p.mode == MODE_PREFILL || c < p.N) {
+    a1 = (c + 1) * p.L;
+  } else {
+    a1 = (c - p.N) * p.L;
+    b0 = c * p.L;
+    b1 = b0 + p.L;
+  }
+}
+
+// Queries that see key j: [a0, a1) and [b0, b1).
+__device__ __forceinline__ void k_queries(const BwdParams& p, int j, int& a0, int& a1, int& b0,
+                                          int& b1) {
+  const int c = j / p.L;
+  b0 = b1 = 0;
+  a0 = c * p.L;
+  if (p.mode == MODE_PREFILL) {
+    a1 = p.S;
+  } else if (c < p.N) {
+    a1 = p.N * p.L;
+    b0 = (p.N + c + 1) * p.L;
+    b1 = 2 * p.N * p.L;
+  } else {
+    a1 = a0 + p.L;
+  }
+}
+
+// Does any query of tile qt see any key of tile kt?
+__device__ __forceinline__ bool pair_visible(const BwdParams& p, int qt, int kt) {
+  const int q0 = qt * BT, q1 = min(q0 + BT, p.S);
+  const int k0 = kt * BT, k1 = min(k0 + BT, p.S);
+  for (int c = q0 / p.L; c <= (q1 - 1) / p.L; ++c) {
+    int a0, a1, b0, b1;
+    q_keys(p, c * p.L, a0, a1, b0, b1);
+    if ((a0 < k1 && k0 < a1) || (b0 < k1 && k0 < b1)) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ uint32_t bits_in(int lo, int hi) {
+  lo = max(lo, 0);
+  hi = min(hi, 32);
+  if (hi <= lo) return 0u;
+  const uint32_t up = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  return up & ~((1u << lo) - 1u);
+}
+
+__device__ __forceinline__ void bdrain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer() - t0 > DZ_WAIT_NS) return;
+  }
+}
+
+// Rotary position of token s (noisy teacher-forcing tokens take clean positions).
+__device__ __forceinline__ void bpos(const BwdParams& p, int s, int& t, int& h, int& w) {
+  token_pos(p.geom, p.period > 0 ? s % p.period : s, 0, t, h, w);
+}
+
+// fp32 row chunk of 32 gradient features (pairs 16*c .. 16*c + 15) turned back by
+// -theta, scaled, rounded to bf16 and stored (16-byte stores).
+__device__ __forceinline__ void store_rotated_back(__nv_bfloat16* dst, const uint32_t (&v)[32],
+                                                   const RopeTables& r, int c, int t, int h, int w,
+                                                   float scale) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float2 cs = __ldg(r.tab + rope_index(r, 16 * c + i, t, h, w));
+    const float x0 = __uint_as_float(v[2 * i]) * scale, x1 = __uint_as_float(v[2 * i + 1]) * scale;
+    const float y0 = __fmaf_rn(x0, cs.x, __fmul_rn(x1, cs.y));
+    const float y1 = __fmaf_rn(x1, cs.x, -__fmul_rn(x0, cs.y));
+    pk[i] = pack_bf16x2(y0, y1);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) d[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+}
+
+__device__ __forceinline__ void tile_load(uint8_t* dst, const CUtensorMap* m, uint64_t* bar,
+                                          int h, int row, int b) {
+  tma_load_4d(dst, m, bar, 0, h, row, b);
+  tma_load_4d(dst + BHALF, m, bar, 64, h, row, b);
+}
+
+// K-major A and B (SS) product over the 128 head dims: D[128 x 128] = A B^T.
+__device__ __forceinline__ void mma_kmajor(uint32_t d, uint32_t a_lo, uint32_t b_lo,
+                                           uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < HEAD_DIM / 16; ++kk) {
+    const uint32_t off = ((kk >> 2) * BHALF + (kk & 3) * 32) >> 4;
+    mma_ss(d, desc_join(a_lo + off), desc_join(b_lo + off), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// D[128 x 128] (+)= A B with A (bf16, 128 rows x 128 K) in TMEM at column a and B
+// (128 K rows x 128 dims) MN-major in shared memory.
+__device__ __forceinline__ void mma_tmem_a(uint32_t d, uint32_t a, uint32_t b_lo, uint32_t idesc,
+                                           bool acc) {
+#pragma unroll
+  for (int kk = 0; kk < BT / 16; ++kk)
+    mma_ts(d, a + kk * 8, desc_join(b_lo + ((kk * 16 * 128) >> 4)), idesc,
+           (acc || kk > 0) ? 1u : 0u);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// dQ: one CTA per (batch, head, query tile).  TMEM: S [0,128) (dS bf16 over its
+// first 64 columns), dP [128,256), dQ [256,384).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + BSM_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BSM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + BSM_MISC + 4);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x % p.n_tiles;
+  const int bh = blockIdx.x / p.n_tiles;
+  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  const int q0 = qt * BT;
+
+  if (tid == 0) {
+    mbar_init(&bar[BB_FIX], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[BB_FULL + s], 1);
+      mbar_init(&bar[BB_EMPTY + s], 1);
+    }
+    mbar_init(&bar[BB_SDP], 1);
+    mbar_init(&bar[BB_READY], 128);
+    mbar_init(&bar[BB_ACC], 1);
+    mbar_init(&bar[BB_DRAIN], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(&bar[BB_FIX], 2 * BTILE);
+      tile_load(smem + BSM_FIXED0, &p.tm_q, &bar[BB_FIX], h, q0, b);
+      tile_load(smem + BSM_FIXED1, &p.tm_do, &bar[BB_FIX], h, q0, b);
+      uint32_t it = 0;
+      for (int kt = 0; kt < p.n_tiles; ++kt) {
+        if (!pair_visible(p, qt, kt)) continue;
+        const int st = it & 1;
+        if (!mbar_wait(&bar[BB_EMPTY + st], ((it >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        uint8_t* ring = smem + BSM_RING + st * 2 * BTILE;
+        mbar_expect_tx(&bar[BB_FULL + st], 2 * BTILE);
+        tile_load(ring, &p.tm_k, &bar[BB_FULL + st], h, kt * BT, b);
+        tile_load(ring + BTILE, &p.tm_v, &bar[BB_FULL + st], h, kt * BT, b);
+        ++it;
+      }
+      bdrain(&bar[BB_FIX], 0);
+      for (uint32_t j = (it > 2 ? it - 2 : 0); j < it; ++j) bdrain(&bar[BB_FULL + (j & 1)], (j >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_kk = idesc_bf16(BT, BT, false);
+      const uint32_t id_mn = idesc_bf16(BT, HEAD_DIM, true);
+      const uint32_t q_lo = desc_lo(smem_u32(smem + BSM_FIXED0), 16);
+      const uint32_t do_lo = desc_lo(smem_u32(smem + BSM_FIXED1), 16);
+      bool ok = mbar_wait(&bar[BB_FIX], 0, abort_flag, p.status);
+      tc_fence_after();
+      uint32_t it = 0;
+      int pst = 0;
+      for (int kt = 0; ok && kt < p.n_tiles; ++kt) {
+        if (!pair_visible(p, qt, kt)) continue;
+        const int st = it & 1;
+        if (!mbar_wait(&bar[BB_FULL + st], (it >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        if (it > 0) {
+          // dQ += dS K for the previous key tile (dS over S in TMEM)
+          if (!mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t k_mn = desc_lo(smem_u32(smem + BSM_RING + pst * 2 * BTILE), BHALF);
+          mma_tmem_a(tmem + 256, tmem, k_mn, id_mn, it > 1);
+          mma_commit(&bar[BB_EMPTY + pst]);
+        }
+        const uint32_t k_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), 16);
+        const uint32_t v_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE + BTILE), 16);
+        mma_kmajor(tmem, q_lo, k_lo, id_kk);          // S = Q K^T
+        mma_kmajor(tmem + 128, do_lo, v_lo, id_kk);   // dP = dO V^T
+        mma_commit(&bar[BB_SDP]);
+        pst = st;
+        ++it;
+      }
+      if (ok && it > 0 && mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) {
+        tc_fence_after();
+        const uint32_t k_mn = desc_lo(smem_u32(smem + BSM_RING + pst * 2 * BTILE), BHALF);
+        mma_tmem_a(tmem + 256, tmem, k_mn, id_mn, it > 1);
+        mma_commit(&bar[BB_EMPTY + pst]);
+      }
+      mma_commit(&bar[BB_ACC]);
+      mma_commit(&bar[BB_DRAIN]);
+      bdrain(&bar[BB_DRAIN], 0);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    const uint32_t la = static_cast<uint32_t>(32 * quarter) << 16;
+    const int s = q0 + r;
+    const bool valid = s < p.S;
+    const int s_eff = valid ? s : p.S - 1;
+    const size_t vec = static_cast<size_t>(bh) * p.S + s_eff;
+    const float lse2 = p.lse[vec];
+    const float dsum = p.dd[vec];
+    int a0, a1, b0, b1;
+    q_keys(p, s_eff, a0, a1, b0, b1);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int kt = 0; kt < p.n_tiles; ++kt) {
+      if (!pair_visible(p, qt, kt)) continue;
+      if (!mbar_wait(&bar[BB_SDP], it & 1, abort_flag, p.status)) { ok = false; break; }
+      tc_fence_after();
+      const int k0 = kt * BT;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tmem + la + 32 * c, sv);
+        tmem_ld32(tmem + la + 128 + 32 * c, dp);
+        tmem_wait_ld();
+        const int col0 = k0 + 32 * c;
+        const uint32_t keep = bits_in(a0 - col0, a1 - col0) | bits_in(b0 - col0, b1 - col0);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int j = 2 * i + e;
+            const float pr = ((keep >> j) & 1u) ? ex2(__uint_as_float(sv[j]) * p.scale_log2 - lse2) : 0.f;
+            d2[e] = pr * (__uint_as_float(dp[j]) - dsum);
+          }
+          pk[i] = pack_bf16x2(d2[0], d2[1]);
+        }
+        tmem_st16(tmem + la + 16 * c, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar[BB_READY]);
+      ++it;
+    }
+    if (ok && mbar_wait(&bar[BB_ACC], 0, abort_flag, p.status)) {
+      tc_fence_after();
+      int t, hh, w;
+      bpos(p, s_eff, t, hh, w);
+      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(b * p.S + s_eff) * p.H + h) * HEAD_DIM;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + la + 256 + 32 * c, v);
+        tmem_wait_ld();
+        if (it == 0) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = 0u;
+        }
+        if (valid) store_rotated_back(dst + 32 * c, v, p.rope, c, t, hh, w, p.scale);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV: one CTA per (batch, head, key tile).  TMEM: S^T [0,128) (P^T bf16 over
+// its first 64 columns), dP^T [128,256) (dS^T bf16 over its first 64 columns),
+// dV [256,384), dK [384,512).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_constant__ BwdParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + BSM_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BSM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + BSM_MISC + 4);
+  float* sm_vec = reinterpret_cast<float*>(smem + BSM_VEC);  // [2 buffers][lse 128 | D 128]
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kt = blockIdx.x % p.n_tiles;
+  const int bh = blockIdx.x / p.n_tiles;
+  const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+  const int k0 = kt * BT;
+
+  if (tid == 0) {
+    mbar_init(&bar[BB_FIX], 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bar[BB_FULL + s], 1);
+      mbar_init(&bar[BB_EMPTY + s], 1);
+    }
+    mbar_init(&bar[BB_SDP], 1);
+    mbar_init(&bar[BB_READY], 128);
+    mbar_init(&bar[BB_ACC], 1);
+    mbar_init(&bar[BB_DRAIN], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_expect_tx(&bar[BB_FIX], 2 * BTILE);
+      tile_load(smem + BSM_FIXED0, &p.tm_k, &bar[BB_FIX], h, k0, b);
+      tile_load(smem + BSM_FIXED1, &p.tm_v, &bar[BB_FIX], h, k0, b);
+      uint32_t it = 0;
+      for (int qt = 0; qt < p.n_tiles; ++qt) {
+        if (!pair_visible(p, qt, kt)) continue;
+        const int st = it & 1;
+        if (!mbar_wait(&bar[BB_EMPTY + st], ((it >> 1) & 1) ^ 1, abort_flag, p.status)) break;
+        uint8_t* ring = smem + BSM_RING + st * 2 * BTILE;
+        mbar_expect_tx(&bar[BB_FULL + st], 2 * BTILE);
+        tile_load(ring, &p.tm_q, &bar[BB_FULL + st], h, qt * BT, b);
+        tile_load(ring + BTILE, &p.tm_do, &bar[BB_FULL + st], h, qt * BT, b);
+        ++it;
+      }
+      bdrain(&bar[BB_FIX], 0);
+      for (uint32_t j = (it > 2 ? it - 2 : 0); j < it; ++j) bdrain(&bar[BB_FULL + (j & 1)], (j >> 1) & 1);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_kk = idesc_bf16(BT, BT, false);
+      const uint32_t id_mn = idesc_bf16(BT, HEAD_DIM, true);
+      const uint32_t k_lo = desc_lo(smem_u32(smem + BSM_FIXED0), 16);
+      const uint32_t v_lo = desc_lo(smem_u32(smem + BSM_FIXED1), 16);
+      bool ok = mbar_wait(&bar[BB_FIX], 0, abort_flag, p.status);
+      tc_fence_after();
+      uint32_t it = 0;
+      int pst = 0;
+      auto grads = [&](int stage, bool acc) {
+        const uint32_t q_mn = desc_lo(smem_u32(smem + BSM_RING + stage * 2 * BTILE), BHALF);
+        const uint32_t do_mn = desc_lo(smem_u32(smem + BSM_RING + stage * 2 * BTILE + BTILE), BHALF);
+        mma_tmem_a(tmem + 256, tmem, do_mn, id_mn, acc);        // dV += P^T dO
+        mma_tmem_a(tmem + 384, tmem + 128, q_mn, id_mn, acc);   // dK += dS^T Q
+        mma_commit(&bar[BB_EMPTY + stage]);
+      };
+      for (int qt = 0; ok && qt < p.n_tiles; ++qt) {
+        if (!pair_visible(p, qt, kt)) continue;
+        const int st = it & 1;
+        if (!mbar_wait(&bar[BB_FULL + st], (it >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        if (it > 0) {
+          if (!mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          grads(pst, it > 1);
+        }
+        const uint32_t q_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), 16);
+        const uint32_t do_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE + BTILE), 16);
+        mma_kmajor(tmem, k_lo, q_lo, id_kk);          // S^T = K Q^T
+        mma_kmajor(tmem + 128, v_lo, do_lo, id_kk);   // dP^T = V dO^T
+        mma_commit(&bar[BB_SDP]);
+        pst = st;
+        ++it;
+      }
+      if (ok && it > 0 && mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) {
+        tc_fence_after();
+        grads(pst, it > 1);
+      }
+      mma_commit(&bar[BB_ACC]);
+      mma_commit(&bar[BB_DRAIN]);
+      bdrain(&bar[BB_DRAIN], 0);
+    }
+  } else {
+    const int quarter = warp & 3;
+    const int r = 32 * quarter + lane;
+    const int ct = tid - 64;  // 0..127 among the compute threads
+    const uint32_t la = static_cast<uint32_t>(32 * quarter) << 16;
+    const int j = k0 + r;
+    const bool valid = j < p.S;
+    const int j_eff = valid ? j : p.S - 1;
+    int a0, a1, b0, b1;
+    k_queries(p, j_eff, a0, a1, b0, b1);
+    const size_t vbase = static_cast<size_t>(bh) * p.S;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int qt = 0; qt < p.n_tiles; ++qt) {
+      if (!pair_visible(p, qt, kt)) continue;
+      const int q0 = qt * BT;
+      // the query tile's lse and D, one per thread, double-buffered across steps
+      float* vb = sm_vec + (it & 1) * 2 * BT;
+      const int qq = q0 + ct;
+      vb[ct] = qq < p.S ? p.lse[vbase + qq] : 0.f;
+      vb[BT + ct] = qq < p.S ? p.dd[vbase + qq] : 0.f;
+      named_bar_sync(1, 128);
+      if (!mbar_wait(&bar[BB_SDP], it & 1, abort_flag, p.status)) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tmem + la + 32 * c, sv);
+        tmem_ld32(tmem + la + 128 + 32 * c, dp);
+        tmem_wait_ld();
+        const int col0 = q0 + 32 * c;
+        const uint32_t keep = bits_in(a0 - col0, a1 - col0) | bits_in(b0 - col0, b1 - col0);
+        uint32_t pp[16], pd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float pr[2], d2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int jj = 2 * i + e;
+            const int col = 32 * c + jj;
+            pr[e] = ((keep >> jj) & 1u) ? ex2(__uint_as_float(sv[jj]) * p.scale_log2 - vb[col]) : 0.f;
+            d2[e] = pr[e] * (__uint_as_float(dp[jj]) - vb[BT + col]);
+          }
+          pp[i] = pack_bf16x2(pr[0], pr[1]);
+          pd[i] = pack_bf16x2(d2[0], d2[1]);
+        }
+        tmem_st16(tmem + la + 16 * c, pp);
+        tmem_st16(tmem + la + 128 + 16 * c, pd);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar[BB_READY]);
+      ++it;
+    }
+    if (ok && mbar_wait(&bar[BB_ACC], 0, abort_flag, p.status)) {
+      tc_fence_after();
+      int t, hh, w;
+      bpos(p, j_eff, t, hh, w);
+      const size_t row = (static_cast<size_t>(b * p.S + j_eff) * p.H + h) * HEAD_DIM;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + la + 256 + 32 * c, v);
+        tmem_wait_ld();
+        if (it == 0) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (valid) {
+          uint4* d = reinterpret_cast<uint4*>(p.dv + row + 32 * c);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            d[e] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                              pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                              pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                              pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+        }
+      }
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + la + 384 + 32 * c, v);
+        tmem_wait_ld();
+        if (it == 0) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (valid) store_rotated_back(p.dk + row + 32 * c, v, p.rope, c, t, hh, w, p.scale);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D = rowsum(dO * O) per (batch, token, head) row, fp32, into [B][H][S].
+__global__ void bwd_rowdot_kernel(const uint4* dout, const uint4* out, float* dd, int B, int S,
+                                  int H) {
+  const long long row = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (row >= static_cast<long long>(B) * S * H) return;
+  const uint4* a = dout + row * (HEAD_DIM / 8);
+  const uint4* c = out + row * (HEAD_DIM / 8);
+  float acc = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < HEAD_DIM / 8; ++i) {
+    const uint4 x = a[i], y = c[i];
+    const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const __nv_bfloat162 xa = *reinterpret_cast<const __nv_bfloat162*>(&xs[k]);
+      const __nv_bfloat162 ya = *reinterpret_cast<const __nv_bfloat162*>(&ys[k]);
+      acc = __fmaf_rn(__low2float(xa), __low2float(ya), acc);
+      acc = __fmaf_rn(__high2float(xa), __high2float(ya), acc);
+    }
+  }
+  const long long h = row % H;
+  const long long bs = row / H;
+  const long long b = bs / S, s = bs - b * S;
+  dd[(b * H + h) * S + s] = acc;
+}
+
+cudaError_t launch_backward(const BwdLaunch& a, cudaStream_t stream) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         BSMEM_BYTES);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BSMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  const long long rows = static_cast<long long>(a.B) * a.S * a.H;
+  bwd_rowdot_kernel<<<static_cast<unsigned>((rows + 255) / 256), 256, 0, stream>>>(
+      static_cast<const uint4*>(a.dout), static_cast<const uint4*>(a.out), a.dd, a.B, a.S, a.H);
+  BwdParams p;
+  p.tm_q = a.tm_q;
+  p.tm_k = a.tm_k;
+  p.tm_v = a.tm_v;
+  p.tm_do = a.tm_do;
+  p.lse = a.lse;
+  p.dd = a.dd;
+  p.dq = static_cast<__nv_bfloat16*>(a.dq);
+  p.dk = static_cast<__nv_bfloat16*>(a.dk);
+  p.dv = static_cast<__nv_bfloat16*>(a.dv);
+  p.rope = a.rope;
+  p.geom = a.geom;
+  p.mode = a.mode;
+  p.L = a.geom.L;
+  p.N = a.N;
+  p.S = a.S;
+  p.B = a.B;
+  p.H = a.H;
+  p.n_tiles = (a.S + BT - 1) / BT;
+  p.period = a.mode == MODE_TEACHER_FORCING ? a.N * a.geom.L : 0;
+  p.scale = 1.f / sqrtf(static_cast<float>(HEAD_DIM));
+  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));
+  p.status = a.status;
+  const unsigned grid = static_cast<unsigned>(a.B * a.H * p.n_tiles);
+  bwd_dq_kernel<<<grid, BTHREADS, BSMEM_BYTES, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dkv_kernel<<<grid, BTHREADS, BSMEM_BYTES, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace dz

@@ -157,6 +157,7 @@ cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const Chu
 struct AttnLaunch {
   CUtensorMap tm_q, tm_k, tm_v, tm_ck, tm_cv;
   void* out;
+  float* lse;  // null, or fp32 [B][H][Sq]: m + log2(l) of each query row's softmax
   float* ws;
   int* counters;
   int* status;
@@ -199,6 +200,20 @@ struct QkvLaunch {
 // Capacity (float2 entries) of the projection kernel's shared-memory rotary table.
 constexpr int QKV_ROPE_STAGE_MAX = 4096;
 cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream);
+
+// Backward of the prefill / teacher-forcing attention; see dz_bwd.cu.
+struct BwdLaunch {
+  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // rotated q, rotated k, v, dO (4-D, 128-row boxes)
+  const void *out, *dout;               // bf16 [B][S][H][128]
+  const float* lse;                     // [B][H][S] from the forward (log2 domain)
+  float* dd;                            // workspace [B][H][S]: rowsum(dO * O)
+  void *dq, *dk, *dv;                   // bf16 [B][S][H][128]
+  RopeTables rope;
+  ChunkGeom geom;
+  int mode, N, S, B, H;
+  int* status;
+};
+cudaError_t launch_backward(const BwdLaunch& a, cudaStream_t stream);
 
 // Workspace (in floats) one partial-result slot needs: Q_TILES * TILE_M rows of
 // HEAD_DIM accumulators plus (m, l) per row.

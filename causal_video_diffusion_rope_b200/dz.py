@@ -34,7 +34,8 @@ DZ_MODE_ROTATED = 0x100  # flag: q and the call's own k are already rotated
 EXPORTS = [
     "dz_attn_create", "dz_attn_destroy", "dz_rope3d", "dz_chunk_attn_forward",
     "dz_kvcache_append", "dz_kvcache_replace", "dz_attn_sync_status", "dz_status_string",
-    "dz_chunk_attn_forward_noalloc", "dz_qkv_rope",
+    "dz_chunk_attn_forward_noalloc", "dz_qkv_rope", "dz_chunk_attn_forward_lse",
+    "dz_chunk_attn_backward",
 ]
 
 
@@ -99,6 +100,10 @@ def load() -> ctypes.CDLL:
     lib.dz_kvcache_replace.argtypes = [vp, ctypes.POINTER(dz_kvcache), i32, vp, vp, vp]
     lib.dz_qkv_rope.argtypes = [vp, vp, vp, i32, i32, i32, ctypes.POINTER(dz_chunk_layout), i32,
                                 vp, vp, vp, ctypes.POINTER(dz_kvcache), vp]
+    lib.dz_chunk_attn_forward_lse.argtypes = [vp, vp, vp, vp, ctypes.POINTER(dz_chunk_layout),
+                                              vp, vp, vp]
+    lib.dz_chunk_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp,
+                                           ctypes.POINTER(dz_chunk_layout), vp, vp, vp, vp]
     lib.dz_attn_sync_status.argtypes = [vp, vp]
     lib.dz_status_string.argtypes = [ctypes.c_int]
     lib.dz_status_string.restype = ctypes.c_char_p
@@ -216,6 +221,22 @@ def dz_qkv_rope(handle: int, x, w, B: int, S: int, d_model: int, layout: dz_chun
     _check(load().dz_qkv_rope(handle, _ptr(x), _ptr(w), B, S, d_model, ctypes.byref(layout),
                               first_chunk, _ptr(q_out), _ptr(k_out), _ptr(v_out), cptr,
                               _stream(stream)), "dz_qkv_rope")
+
+
+def dz_chunk_attn_forward_lse(handle: int, q, k, v, layout: dz_chunk_layout, out, lse,
+                              stream=None) -> None:
+    """Training-form forward: also writes each query row's log2 softmax normaliser."""
+    _check(load().dz_chunk_attn_forward_lse(handle, _ptr(q), _ptr(k), _ptr(v),
+                                            ctypes.byref(layout), _ptr(out), _ptr(lse),
+                                            _stream(stream)), "dz_chunk_attn_forward_lse")
+
+
+def dz_chunk_attn_backward(handle: int, q, k, v, out, dout, lse, layout: dz_chunk_layout,
+                           dq, dk, dv, stream=None) -> None:
+    """Gradients of sum(dout * out) with respect to the unrotated q, k and v."""
+    _check(load().dz_chunk_attn_backward(handle, _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
+                                         _ptr(lse), ctypes.byref(layout), _ptr(dq), _ptr(dk),
+                                         _ptr(dv), _stream(stream)), "dz_chunk_attn_backward")
 
 
 def dz_attn_sync_status(handle: int, stream=None) -> None:

@@ -212,6 +212,36 @@ dz_status dz_kvcache_append(dz_attn_t handle, dz_kvcache* cache, const void* k, 
 dz_status dz_kvcache_replace(dz_attn_t handle, dz_kvcache* cache, int32_t chunk_index,
                              const void* k, const void* v, void* stream);
 
+/* Training form of the attention: dz_chunk_attn_forward for DZ_MODE_PREFILL or
+ * DZ_MODE_TEACHER_FORCING (no cache), which also writes, for every query row,
+ * the log2-domain normaliser of its softmax,
+ *   lse[b][h][s] = log2( sum over visible keys j of 2^(S_sj * log2(e)) ),
+ *   S = (R q)(R k)^T / sqrt(128) in fp32,
+ * as fp32 [B][H][Sq] (16-byte aligned).  dz_chunk_attn_backward consumes it.
+ * Errors: as dz_chunk_attn_forward, and DZ_ERR_UNSUPPORTED for other modes. */
+dz_status dz_chunk_attn_forward_lse(dz_attn_t handle, const void* q, const void* k, const void* v,
+                                    const dz_chunk_layout* layout, void* out, void* lse,
+                                    void* stream);
+
+/* Backward of the prefill / teacher-forcing attention (the training form of the
+ * chunk mask: hyper.ai summary of the paper, "方法" (teacher forcing); the
+ * walkthrough's training objective, Fig. 14).  Given the forward's inputs
+ * q, k, v (unrotated), its output `out`, its `lse` (dz_chunk_attn_forward_lse)
+ * and the output gradient `dout` (all bf16 [B][S][H][128] but lse), writes the
+ * gradients of sum(dout * out) with respect to q, k and v:
+ *   dv = P^T dout,  dP = dout v^T,  dS = P * (dP - rowsum(dout * out)),
+ *   dq = R^T (dS (R k)) / sqrt(128),  dk = R^T (dS^T (R q)) / sqrt(128),
+ * accumulated in fp32 and rounded once to bf16 (dq, dk, dv [B][S][H][128]).
+ * Uses the handle's rotation workspace (prerotate_tokens >= S) and its split
+ * workspace (B * H * S floats); calls on one handle must not overlap.
+ * Errors: DZ_ERR_INVALID_ARG, DZ_ERR_ALIGNMENT, DZ_ERR_SHAPE, DZ_ERR_UNSUPPORTED
+ * (DECODE or CROSS), DZ_ERR_CAPACITY (batch, tokens or workspaces beyond the
+ * handle), DZ_ERR_CUDA. */
+dz_status dz_chunk_attn_backward(dz_attn_t handle, const void* q, const void* k, const void* v,
+                                 const void* out, const void* dout, const void* lse,
+                                 const dz_chunk_layout* layout, void* dq, void* dk, void* dv,
+                                 void* stream);
+
 /* QKV projection with the rotary embedding and the KV-cache append fused into
  * one GEMM ("DreamZero (WAM) 模型架构", §2.3 block diagram: the causal
  * self-attention of each DiT block takes the normalised, modulated hidden
