@@ -557,6 +557,76 @@ def run_qkv(args, rank: int, world: int, local_rank: int, config: dict):
     print(json.dumps(line), flush=True)
 
 
+BWD_METRIC = ("chunk-causal attention backward TFLOP/s (dq, dk, dv; algorithmic 2.5x the "
+              "forward's visible-pair FLOP) and % of B200 BF16 peak; \u00b5s per call")
+
+
+def run_bwd(args, rank: int, world: int, local_rank: int, config: dict):
+    """Times dz_chunk_attn_backward on a prefill / teacher-forcing workload."""
+    import torch
+    from causal_video_diffusion_rope_b200 import dz
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    lay = w.layout
+    if lay.mode not in (synth.MODE_PREFILL, synth.MODE_TEACHER_FORCING):
+        raise SystemExit("--op bwd needs a prefill or teacher-forcing workload (e.g. --workload 3)")
+    B, H, D, S = lay.batch, w.heads, w.head_dim, lay.q_len
+    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=S,
+                                       prerotate_tokens=S))
+    dl = dz.layout_from(lay)
+    rng = np.random.default_rng(1000 * rank + 7)
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    q, k, v, dout = (dev_bf16(synth.normal_bf16(rng, (B, S, H, D))) for _ in range(4))
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        dz.dz_chunk_attn_forward_lse(h, q, k, v, dl, out, lse, stream)
+
+    def call(i):
+        dz.dz_chunk_attn_backward(h, q, k, v, out, dout, lse, dl, dq, dk, dv, stream)
+
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    ms, clocks = time_graph(stream, call, args.steps, args.warmup, world, dev, sampler)
+    dz.dz_attn_sync_status(h, stream)
+    ms_per_step = ms / args.steps
+    flops = 2.5 * step_flops(w)
+
+    def e2e_call(di, do):
+        dz.dz_chunk_attn_backward(h, di["q"], di["k"], di["v"], di["out"], di["dout"], di["lse"],
+                                  dl, do["dq"], do["dk"], do["dv"], stream)
+
+    e2e = e2e_pipelined(dev, stream, {"q": q, "k": k, "v": v, "out": out, "dout": dout, "lse": lse},
+                        {"dq": dq, "dk": dk, "dv": dv}, e2e_call, max(3, min(args.steps, 20)), world)
+    e2e["value"] = round(job_throughput(flops, e2e.pop("steps_done"), world, e2e.pop("ms")), 3)
+    dz.dz_attn_sync_status(h, stream)
+    dz.dz_attn_destroy(h)
+    if rank != 0:
+        return
+    peak_tf, _, peak_kind = measured_peaks()
+    per_gpu = flops / (ms_per_step * 1e-3) / 1e12
+    line = {"metric": BWD_METRIC, "value": round(job_throughput(flops, args.steps, world, ms), 3),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6), "us_per_call": round(ms_per_step * 1e3, 3),
+            "pct_of_bf16_peak": round(100 * per_gpu / peak_tf, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (q, k, v, dO ~ N(0,1))",
+            "config": dict(config, op="backward", flop_per_step=flops,
+                           l2=f"q, k, v, out, dO: {5 * B * S * H * D * 2 / 2**20:.0f} MiB > 126 MB L2",
+                           parallelism=f"dp{world} (independent replicas of the call)"),
+            "roofline": {"bound": "tensor", "achieved": round(per_gpu, 2), "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": round(per_gpu / peak_tf, 4), "traffic": None,
+                         "peak_kind": f"{peak_kind} bf16 (burst)",
+                         "kernel": "bwd_dq_kernel + bwd_dkv_kernel"},
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": 4 * args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -565,8 +635,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle CPU work for the cpu_baseline field")
-    ap.add_argument("--op", default="attn", choices=["attn", "qkv"],
-                    help="attn: the chunk-causal attention call; qkv: the fused projection")
+    ap.add_argument("--op", default="attn", choices=["attn", "qkv", "bwd"],
+                    help="attn: the chunk-causal attention call; qkv: the fused projection; "
+                         "bwd: the backward of a prefill / teacher-forcing call")
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
                     choices=range(len(synth.WORKLOADS)),
                     help="workload index (default: the single-layer inference step)")
@@ -586,7 +657,7 @@ def main():
               "rope": "3d t/h/w 22/21/21 base 1e4; q and the chunk's k rotated once per call",
               "flop_per_step": step_flops(w)}
 
-    if args.op == "qkv":
+    if args.op in ("qkv", "bwd"):
         if args.impl == "reference":
             if rank == 0:
                 print(json.dumps({"impl": "reference", "unavailable": "the reference arm times "
@@ -596,7 +667,7 @@ def main():
         if world > 1:
             import datetime
             dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        run_qkv(args, rank, world, local_rank, config)
+        (run_qkv if args.op == "qkv" else run_bwd)(args, rank, world, local_rank, config)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
