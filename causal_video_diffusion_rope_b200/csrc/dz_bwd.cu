@@ -17,9 +17,14 @@
 //                   that see it, S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
 //                   written as bf16 over them in TMEM, then dV += P^T dO and
 //                   dK += dS^T Q.
-// Each has a TMA warp (2-stage ring of the streamed tiles), an MMA warp and four
-// warps that own one TMEM lane (one tile row) per thread.  The rotation back
-// (R^T) and the 1/sqrt(128) are applied to the fp32 accumulators in the epilogue.
+// Each has a TMA warp (2-stage ring of the streamed tiles), an MMA warp and eight
+// compute warps: two per TMEM lane quarter, one thread per tile row, each of the
+// two taking 32 of a half-tile's 64 columns.  A streamed tile is taken in two
+// halves of 64 rows with two TMEM buffers, so that the products of one half run
+// while the compute warps turn the other half's scores into bf16 operands.  Each
+// thread writes its bf16 operands over its own fp32 columns, so a half's operand
+// occupies columns [0, 16) and [32, 48) of its region (see mma_tmem_a64).  The rotation back (R^T) and the 1/sqrt(128) are applied to the fp32
+// accumulators in the epilogue.
 #include "dz_internal.cuh"
 #include "dz_ptx.cuh"
 
@@ -28,7 +33,8 @@ namespace dz {
 namespace {
 
 constexpr int BT = 128;                            // rows of a query or key tile
-constexpr int BTHREADS = 192;                      // warp 0 TMA, 1 MMA, 2-5 compute
+constexpr int BTHREADS = 320;                      // warp 0 TMA, 1 MMA, 2-9 compute
+constexpr int BCOMPUTE = BTHREADS - 64;            // two warps per TMEM lane quarter
 constexpr int BTILE = BT * HEAD_DIM * 2;           // 32 KiB
 constexpr int BHALF = BTILE / 2;                   // 64 dims x 128 rows
 constexpr int BSM_FIXED0 = 0;                      // resident tile 0 (Q or K)
@@ -44,12 +50,13 @@ enum {
   BB_FIX = 0,         // resident tiles landed
   BB_FULL = 1,        // [2] ring stage landed
   BB_EMPTY = 3,       // [2] ring stage consumed
-  BB_SDP = 5,         // S and dP (or their transposes) in TMEM
-  BB_READY = 6,       // compute warps wrote the bf16 operands (128 arrivals)
-  BB_ACC = 7,         // accumulators final
-  BB_DRAIN = 8,
-  BB_COUNT = 9
+  BB_SDP = 5,         // [2] S and dP (or their transposes) of a half in TMEM buffer u
+  BB_READY = 7,       // [2] compute warps wrote the half's bf16 operands (128 arrivals)
+  BB_ACC = 9,         // accumulators final
+  BB_DRAIN = 10,
+  BB_COUNT = 11
 };
+static_assert(BB_COUNT * 8 <= 256, "barrier area");
 
 struct __align__(64) BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;  // rotated q, rotated k, v, dO: (128, H, S, B)
@@ -155,7 +162,8 @@ __device__ __forceinline__ void tile_load(uint8_t* dst, const CUtensorMap* m, ui
   tma_load_4d(dst + BHALF, m, bar, 64, h, row, b);
 }
 
-// K-major A and B (SS) product over the 128 head dims: D[128 x 128] = A B^T.
+// K-major A and B (SS) product over the 128 head dims: D[128 x N] = A B^T (N set
+// by idesc; b_lo may point at a later row of the B tile).
 __device__ __forceinline__ void mma_kmajor(uint32_t d, uint32_t a_lo, uint32_t b_lo,
                                            uint32_t idesc) {
 #pragma unroll
@@ -165,15 +173,18 @@ __device__ __forceinline__ void mma_kmajor(uint32_t d, uint32_t a_lo, uint32_t b
   }
 }
 
-// D[128 x 128] (+)= A B with A (bf16, 128 rows x 128 K) in TMEM at column a and B
-// (128 K rows x 128 dims) MN-major in shared memory.
-__device__ __forceinline__ void mma_tmem_a(uint32_t d, uint32_t a, uint32_t b_lo, uint32_t idesc,
-                                           bool acc) {
+// D[128 x 128] (+)= A B with A (bf16, 128 rows x 64 K) in TMEM and B (64 K rows x
+// 128 dims) MN-major in shared memory.  A's K columns 0-31 sit at TMEM columns
+// [a, a + 16) and 32-63 at [a + 32, a + 48) (one half per compute warp group).
+__device__ __forceinline__ void mma_tmem_a64(uint32_t d, uint32_t a, uint32_t b_lo, uint32_t idesc,
+                                             bool acc) {
 #pragma unroll
-  for (int kk = 0; kk < BT / 16; ++kk)
-    mma_ts(d, a + kk * 8, desc_join(b_lo + ((kk * 16 * 128) >> 4)), idesc,
+  for (int kk = 0; kk < 64 / 16; ++kk)
+    mma_ts(d, a + (kk >> 1) * 32 + (kk & 1) * 8, desc_join(b_lo + ((kk * 16 * 128) >> 4)), idesc,
            (acc || kk > 0) ? 1u : 0u);
 }
+
+constexpr uint32_t HALF_ROWS_OFF = (64 * 128) >> 4;  // 64 rows of 128 bytes, in 16-byte units
 
 }  // namespace
 
@@ -200,8 +211,10 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
       mbar_init(&bar[BB_FULL + s], 1);
       mbar_init(&bar[BB_EMPTY + s], 1);
     }
-    mbar_init(&bar[BB_SDP], 1);
-    mbar_init(&bar[BB_READY], 128);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bar[BB_SDP + u], 1);
+      mbar_init(&bar[BB_READY + u], BCOMPUTE);
+    }
     mbar_init(&bar[BB_ACC], 1);
     mbar_init(&bar[BB_DRAIN], 1);
     *abort_flag = 0;
@@ -237,40 +250,46 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_kk = idesc_bf16(BT, BT, false);
+      const uint32_t id_n64 = idesc_bf16(BT, 64, false);
       const uint32_t id_mn = idesc_bf16(BT, HEAD_DIM, true);
       const uint32_t q_lo = desc_lo(smem_u32(smem + BSM_FIXED0), 16);
       const uint32_t do_lo = desc_lo(smem_u32(smem + BSM_FIXED1), 16);
       bool ok = mbar_wait(&bar[BB_FIX], 0, abort_flag, p.status);
       tc_fence_after();
-      uint32_t it = 0;
-      int pst = 0;
+      // half-step j = 2 * (key tile ordinal) + half; TMEM buffer = half
+      auto issue_dq = [&](uint32_t jj) {  // dQ += dS K over the 64 keys of half-step jj
+        const int hf = jj & 1, st = (jj >> 1) & 1;
+        const uint32_t k_mn = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), BHALF);
+        mma_tmem_a64(tmem + 256, tmem + 128 * hf, k_mn + hf * HALF_ROWS_OFF, id_mn, jj > 0);
+        if (hf == 1) mma_commit(&bar[BB_EMPTY + st]);
+      };
+      uint32_t t = 0;  // visible key tiles so far
       for (int kt = 0; ok && kt < p.n_tiles; ++kt) {
         if (!pair_visible(p, qt, kt)) continue;
-        const int st = it & 1;
-        if (!mbar_wait(&bar[BB_FULL + st], (it >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        if (it > 0) {
-          // dQ += dS K for the previous key tile (dS over S in TMEM)
-          if (!mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t k_mn = desc_lo(smem_u32(smem + BSM_RING + pst * 2 * BTILE), BHALF);
-          mma_tmem_a(tmem + 256, tmem, k_mn, id_mn, it > 1);
-          mma_commit(&bar[BB_EMPTY + pst]);
-        }
+        const int st = t & 1;
         const uint32_t k_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), 16);
         const uint32_t v_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE + BTILE), 16);
-        mma_kmajor(tmem, q_lo, k_lo, id_kk);          // S = Q K^T
-        mma_kmajor(tmem + 128, do_lo, v_lo, id_kk);   // dP = dO V^T
-        mma_commit(&bar[BB_SDP]);
-        pst = st;
-        ++it;
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t jj = 2 * t + hf;
+          if (jj >= 2) {  // buffer hf is free once half-step jj - 2 is turned into dS
+            if (!mbar_wait(&bar[BB_READY + hf], ((jj - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            issue_dq(jj - 2);
+          }
+          if (hf == 0) {  // the key tile (waited after the previous tile's dQ went out)
+            if (!mbar_wait(&bar[BB_FULL + st], (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+          }
+          mma_kmajor(tmem + 128 * hf, q_lo, k_lo + hf * HALF_ROWS_OFF, id_n64);        // S
+          mma_kmajor(tmem + 128 * hf + 64, do_lo, v_lo + hf * HALF_ROWS_OFF, id_n64);  // dP
+          mma_commit(&bar[BB_SDP + hf]);
+        }
+        ++t;
       }
-      if (ok && it > 0 && mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) {
+      for (uint32_t jj = (2 * t >= 2 ? 2 * t - 2 : 0); ok && jj < 2 * t; ++jj) {
+        if (!mbar_wait(&bar[BB_READY + (jj & 1)], (jj >> 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
-        const uint32_t k_mn = desc_lo(smem_u32(smem + BSM_RING + pst * 2 * BTILE), BHALF);
-        mma_tmem_a(tmem + 256, tmem, k_mn, id_mn, it > 1);
-        mma_commit(&bar[BB_EMPTY + pst]);
+        issue_dq(jj);
       }
       mma_commit(&bar[BB_ACC]);
       mma_commit(&bar[BB_DRAIN]);
@@ -278,6 +297,7 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
     }
   } else {
     const int quarter = warp & 3;
+    const int cg = (warp - 2) >> 2;  // column group: columns [32 cg, 32 cg + 32) of a half
     const int r = 32 * quarter + lane;
     const uint32_t la = static_cast<uint32_t>(32 * quarter) << 16;
     const int s = q0 + r;
@@ -288,20 +308,21 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
     const float dsum = p.dd[vec];
     int a0, a1, b0, b1;
     q_keys(p, s_eff, a0, a1, b0, b1);
-    uint32_t it = 0;
+    uint32_t it = 0;  // visible key tiles so far
     bool ok = true;
-    for (int kt = 0; kt < p.n_tiles; ++kt) {
+    for (int kt = 0; ok && kt < p.n_tiles; ++kt) {
       if (!pair_visible(p, qt, kt)) continue;
-      if (!mbar_wait(&bar[BB_SDP], it & 1, abort_flag, p.status)) { ok = false; break; }
-      tc_fence_after();
       const int k0 = kt * BT;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t hs = 2 * it + hf;  // half-step
+        if (!mbar_wait(&bar[BB_SDP + hf], (hs >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t col = 128 * hf + 32 * cg;
         uint32_t sv[32], dp[32];
-        tmem_ld32(tmem + la + 32 * c, sv);
-        tmem_ld32(tmem + la + 128 + 32 * c, dp);
+        tmem_ld32(tmem + la + col, sv);
+        tmem_ld32(tmem + la + col + 64, dp);
         tmem_wait_ld();
-        const int col0 = k0 + 32 * c;
+        const int col0 = k0 + 64 * hf + 32 * cg;
         const uint32_t keep = bits_in(a0 - col0, a1 - col0) | bits_in(b0 - col0, b1 - col0);
         uint32_t pk[16];
 #pragma unroll
@@ -310,16 +331,16 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int j = 2 * i + e;
-            const float pr = ((keep >> j) & 1u) ? ex2(__uint_as_float(sv[j]) * p.scale_log2 - lse2) : 0.f;
-            d2[e] = pr * (__uint_as_float(dp[j]) - dsum);
+            const float pe = ex2(__uint_as_float(sv[j]) * p.scale_log2 - lse2);
+            d2[e] = ((keep >> j) & 1u) ? pe * (__uint_as_float(dp[j]) - dsum) : 0.f;
           }
           pk[i] = pack_bf16x2(d2[0], d2[1]);
         }
-        tmem_st16(tmem + la + 16 * c, pk);
+        tmem_st16(tmem + la + col, pk);  // dS over this thread's own S columns
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar[BB_READY + hf]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar[BB_READY]);
       ++it;
     }
     if (ok && mbar_wait(&bar[BB_ACC], 0, abort_flag, p.status)) {
@@ -328,13 +349,13 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
       bpos(p, s_eff, t, hh, w);
       __nv_bfloat16* dst = p.dq + (static_cast<size_t>(b * p.S + s_eff) * p.H + h) * HEAD_DIM;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 2 * cg; c < 2 * cg + 2; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem + la + 256 + 32 * c, v);
         tmem_wait_ld();
         if (it == 0) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = 0u;
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
         }
         if (valid) store_rotated_back(dst + 32 * c, v, p.rope, c, t, hh, w, p.scale);
       }
@@ -375,8 +396,10 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
       mbar_init(&bar[BB_FULL + s], 1);
       mbar_init(&bar[BB_EMPTY + s], 1);
     }
-    mbar_init(&bar[BB_SDP], 1);
-    mbar_init(&bar[BB_READY], 128);
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bar[BB_SDP + u], 1);
+      mbar_init(&bar[BB_READY + u], BCOMPUTE);
+    }
     mbar_init(&bar[BB_ACC], 1);
     mbar_init(&bar[BB_DRAIN], 1);
     *abort_flag = 0;
@@ -412,42 +435,48 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_kk = idesc_bf16(BT, BT, false);
+      const uint32_t id_n64 = idesc_bf16(BT, 64, false);
       const uint32_t id_mn = idesc_bf16(BT, HEAD_DIM, true);
       const uint32_t k_lo = desc_lo(smem_u32(smem + BSM_FIXED0), 16);
       const uint32_t v_lo = desc_lo(smem_u32(smem + BSM_FIXED1), 16);
       bool ok = mbar_wait(&bar[BB_FIX], 0, abort_flag, p.status);
       tc_fence_after();
-      uint32_t it = 0;
-      int pst = 0;
-      auto grads = [&](int stage, bool acc) {
-        const uint32_t q_mn = desc_lo(smem_u32(smem + BSM_RING + stage * 2 * BTILE), BHALF);
-        const uint32_t do_mn = desc_lo(smem_u32(smem + BSM_RING + stage * 2 * BTILE + BTILE), BHALF);
-        mma_tmem_a(tmem + 256, tmem, do_mn, id_mn, acc);        // dV += P^T dO
-        mma_tmem_a(tmem + 384, tmem + 128, q_mn, id_mn, acc);   // dK += dS^T Q
-        mma_commit(&bar[BB_EMPTY + stage]);
+      // half-step j = 2 * (query tile ordinal) + half; TMEM buffer = half
+      auto grads = [&](uint32_t jj) {
+        const int hf = jj & 1, st = (jj >> 1) & 1;
+        const uint32_t q_mn = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), BHALF);
+        const uint32_t do_mn = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE + BTILE), BHALF);
+        mma_tmem_a64(tmem + 256, tmem + 128 * hf, do_mn + hf * HALF_ROWS_OFF, id_mn, jj > 0);      // dV += P^T dO
+        mma_tmem_a64(tmem + 384, tmem + 128 * hf + 64, q_mn + hf * HALF_ROWS_OFF, id_mn, jj > 0);  // dK += dS^T Q
+        if (hf == 1) mma_commit(&bar[BB_EMPTY + st]);
       };
+      uint32_t t = 0;
       for (int qt = 0; ok && qt < p.n_tiles; ++qt) {
         if (!pair_visible(p, qt, kt)) continue;
-        const int st = it & 1;
-        if (!mbar_wait(&bar[BB_FULL + st], (it >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        if (it > 0) {
-          if (!mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
-          grads(pst, it > 1);
-        }
+        const int st = t & 1;
         const uint32_t q_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), 16);
         const uint32_t do_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE + BTILE), 16);
-        mma_kmajor(tmem, k_lo, q_lo, id_kk);          // S^T = K Q^T
-        mma_kmajor(tmem + 128, v_lo, do_lo, id_kk);   // dP^T = V dO^T
-        mma_commit(&bar[BB_SDP]);
-        pst = st;
-        ++it;
+        for (int hf = 0; hf < 2; ++hf) {
+          const uint32_t jj = 2 * t + hf;
+          if (jj >= 2) {
+            if (!mbar_wait(&bar[BB_READY + hf], ((jj - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+            grads(jj - 2);
+          }
+          if (hf == 0) {
+            if (!mbar_wait(&bar[BB_FULL + st], (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+            tc_fence_after();
+          }
+          mma_kmajor(tmem + 128 * hf, k_lo, q_lo + hf * HALF_ROWS_OFF, id_n64);        // S^T
+          mma_kmajor(tmem + 128 * hf + 64, v_lo, do_lo + hf * HALF_ROWS_OFF, id_n64);  // dP^T
+          mma_commit(&bar[BB_SDP + hf]);
+        }
+        ++t;
       }
-      if (ok && it > 0 && mbar_wait(&bar[BB_READY], (it - 1) & 1, abort_flag, p.status)) {
+      for (uint32_t jj = (2 * t >= 2 ? 2 * t - 2 : 0); ok && jj < 2 * t; ++jj) {
+        if (!mbar_wait(&bar[BB_READY + (jj & 1)], (jj >> 1) & 1, abort_flag, p.status)) break;
         tc_fence_after();
-        grads(pst, it > 1);
+        grads(jj);
       }
       mma_commit(&bar[BB_ACC]);
       mma_commit(&bar[BB_DRAIN]);
@@ -455,8 +484,9 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
     }
   } else {
     const int quarter = warp & 3;
+    const int cg = (warp - 2) >> 2;  // column group: columns [32 cg, 32 cg + 32) of a half
     const int r = 32 * quarter + lane;
-    const int ct = tid - 64;  // 0..127 among the compute threads
+    const int ct = tid - 64;         // 0..255 among the compute threads
     const uint32_t la = static_cast<uint32_t>(32 * quarter) << 16;
     const int j = k0 + r;
     const bool valid = j < p.S;
@@ -464,27 +494,29 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
     int a0, a1, b0, b1;
     k_queries(p, j_eff, a0, a1, b0, b1);
     const size_t vbase = static_cast<size_t>(bh) * p.S;
-    uint32_t it = 0;
+    uint32_t it = 0;  // visible query tiles so far
     bool ok = true;
-    for (int qt = 0; qt < p.n_tiles; ++qt) {
+    for (int qt = 0; ok && qt < p.n_tiles; ++qt) {
       if (!pair_visible(p, qt, kt)) continue;
       const int q0 = qt * BT;
-      // the query tile's lse and D, one per thread, double-buffered across steps
+      // the query tile's lse (threads 0-127) and D (128-255), double-buffered across tiles
       float* vb = sm_vec + (it & 1) * 2 * BT;
-      const int qq = q0 + ct;
-      vb[ct] = qq < p.S ? p.lse[vbase + qq] : 0.f;
-      vb[BT + ct] = qq < p.S ? p.dd[vbase + qq] : 0.f;
-      named_bar_sync(1, 128);
-      if (!mbar_wait(&bar[BB_SDP], it & 1, abort_flag, p.status)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      {
+        const int qq = q0 + (ct & (BT - 1));
+        vb[ct] = qq < p.S ? (ct < BT ? p.lse[vbase + qq] : p.dd[vbase + qq]) : 0.f;
+      }
+      named_bar_sync(1, BCOMPUTE);
+      for (int hf = 0; hf < 2; ++hf) {
+        const uint32_t hs = 2 * it + hf;  // half-step
+        if (!mbar_wait(&bar[BB_SDP + hf], (hs >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t col = 128 * hf + 32 * cg;
         uint32_t sv[32], dp[32];
-        tmem_ld32(tmem + la + 32 * c, sv);
-        tmem_ld32(tmem + la + 128 + 32 * c, dp);
+        tmem_ld32(tmem + la + col, sv);
+        tmem_ld32(tmem + la + col + 64, dp);
         tmem_wait_ld();
-        const int col0 = q0 + 32 * c;
-        const uint32_t keep = bits_in(a0 - col0, a1 - col0) | bits_in(b0 - col0, b1 - col0);
+        const int qc = 64 * hf + 32 * cg;  // query column of sv[0] within the tile
+        const uint32_t keep = bits_in(a0 - q0 - qc, a1 - q0 - qc) | bits_in(b0 - q0 - qc, b1 - q0 - qc);
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -492,55 +524,58 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int jj = 2 * i + e;
-            const int col = 32 * c + jj;
-            pr[e] = ((keep >> jj) & 1u) ? ex2(__uint_as_float(sv[jj]) * p.scale_log2 - vb[col]) : 0.f;
-            d2[e] = pr[e] * (__uint_as_float(dp[jj]) - vb[BT + col]);
+            const float pe = ex2(__uint_as_float(sv[jj]) * p.scale_log2 - vb[qc + jj]);
+            pr[e] = ((keep >> jj) & 1u) ? pe : 0.f;
+            d2[e] = pr[e] * (__uint_as_float(dp[jj]) - vb[BT + qc + jj]);
           }
           pp[i] = pack_bf16x2(pr[0], pr[1]);
           pd[i] = pack_bf16x2(d2[0], d2[1]);
         }
-        tmem_st16(tmem + la + 16 * c, pp);
-        tmem_st16(tmem + la + 128 + 16 * c, pd);
+        tmem_st16(tmem + la + col, pp);       // P^T over this thread's own S^T columns
+        tmem_st16(tmem + la + col + 64, pd);  // dS^T over its own dP^T columns
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bar[BB_READY + hf]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bar[BB_READY]);
       ++it;
     }
     if (ok && mbar_wait(&bar[BB_ACC], 0, abort_flag, p.status)) {
       tc_fence_after();
-      int t, hh, w;
-      bpos(p, j_eff, t, hh, w);
       const size_t row = (static_cast<size_t>(b * p.S + j_eff) * p.H + h) * HEAD_DIM;
+      if (cg == 0) {  // dV
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + la + 256 + 32 * c, v);
-        tmem_wait_ld();
-        if (it == 0) {
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + la + 256 + 32 * c, v);
+          tmem_wait_ld();
+          if (it == 0) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
-        }
-        if (valid) {
-          uint4* d = reinterpret_cast<uint4*>(p.dv + row + 32 * c);
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          if (valid) {
+            uint4* d = reinterpret_cast<uint4*>(p.dv + row + 32 * c);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            d[e] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
-                              pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
-                              pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
-                              pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+            for (int e = 0; e < 4; ++e)
+              d[e] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * e]), __uint_as_float(v[8 * e + 1])),
+                                pack_bf16x2(__uint_as_float(v[8 * e + 2]), __uint_as_float(v[8 * e + 3])),
+                                pack_bf16x2(__uint_as_float(v[8 * e + 4]), __uint_as_float(v[8 * e + 5])),
+                                pack_bf16x2(__uint_as_float(v[8 * e + 6]), __uint_as_float(v[8 * e + 7])));
+          }
         }
-      }
+      } else {  // dK, turned back
+        int t, hh, w;
+        bpos(p, j_eff, t, hh, w);
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem + la + 384 + 32 * c, v);
-        tmem_wait_ld();
-        if (it == 0) {
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem + la + 384 + 32 * c, v);
+          tmem_wait_ld();
+          if (it == 0) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          if (valid) store_rotated_back(p.dk + row + 32 * c, v, p.rope, c, t, hh, w, p.scale);
         }
-        if (valid) store_rotated_back(p.dk + row + 32 * c, v, p.rope, c, t, hh, w, p.scale);
       }
     }
   }
