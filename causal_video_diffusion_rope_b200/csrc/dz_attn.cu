@@ -297,45 +297,6 @@ __device__ __forceinline__ float exp_pack(const uint32_t (&v)[32], uint32_t (&pk
   return t.x + t.y;
 }
 
-// 2^x for a pair of arguments on the FMA/ALU pipes instead of the MUFU unit:
-// n = round(x) by adding and subtracting 1.5 * 2^23, f = x - n in [-1/2, 1/2],
-// 2^f by a cubic (coefficients from csrc/fit_exp2.py: a minimax fit in relative
-// error, max 8.4e-5 in fp32 Horner form), then n is added to the exponent
-// field.  Arguments below -125 (masked scores) give exactly 0.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  const float2 xc = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-  const float2 big = make_float2(12582912.f, 12582912.f);
-  const float2 j = fadd2(xc, big);
-  const float2 n = fadd2(j, make_float2(-12582912.f, -12582912.f));
-  const float2 f = ffma2(n, make_float2(-1.f, -1.f), xc);
-  float2 pp = ffma2(make_float2(0.0552129931814347f, 0.0552129931814347f), f,
-                    make_float2(0.24271414047058226f, 0.24271414047058226f));
-  pp = ffma2(pp, f, make_float2(0.6932621602543352f, 0.6932621602543352f));
-  pp = ffma2(pp, f, make_float2(0.999919597990084f, 0.999919597990084f));
-  float2 r;
-  r.x = __int_as_float(__float_as_int(pp.x) + (__float_as_int(j.x) << 23));
-  r.y = __int_as_float(__float_as_int(pp.y) + (__float_as_int(j.y) << 23));
-  r.x = x.x < -125.f ? 0.f : r.x;
-  r.y = x.y < -125.f ? 0.f : r.y;
-  return r;
-}
-
-// exp_pack with every exponential evaluated by exp2_poly2 (FMA pipe).
-__device__ __forceinline__ float exp_pack_poly(const uint32_t (&v)[32], uint32_t (&pk)[32], int off,
-                                               float sl2, float mb) {
-  const float2 sc = make_float2(sl2, sl2), nm = make_float2(-mb, -mb);
-  float2 s2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-  for (int j = 0; j < 16; ++j) {
-    const float2 x = ffma2(make_float2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])), sc, nm);
-    const float2 pp = exp2_poly2(x);
-    s2[j & 1] = fadd2(s2[j & 1], pp);
-    pk[off + j] = pack_bf16x2(pp.x, pp.y);
-  }
-  const float2 t = fadd2(s2[0], s2[1]);
-  return t.x + t.y;
-}
-
 // Rotate row r of a swizzled 128x128 bf16 tile (shared address `tile`) when the
 // pair split (PT, PH, PW) is known at compile time and the row's t-, h- and
 // w-table rows sit in shared memory at addresses tt, th, tw: every table read is
