@@ -74,6 +74,18 @@ def test_calls_reject_null_handle(lib):
         dz.DZ_ERR_INVALID_ARG
     assert lib.dz_attn_sync_status(None, None) == dz.DZ_ERR_INVALID_ARG
     assert lib.dz_attn_destroy(None) == dz.DZ_ERR_INVALID_ARG
+    pre = dz.make_layout(dz.DZ_MODE_PREFILL, 1, 1, 4, 4, 4, 2)
+    assert lib.dz_qkv_rope(None, 16, 16, 1, 20, 128, ctypes.byref(pre), 0, 16, 16, 16, None,
+                           None) == dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_chunk_attn_forward_lse(None, 16, 16, 16, ctypes.byref(pre), 16, 16, None) == \
+        dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_chunk_attn_backward(None, 16, 16, 16, 16, 16, 16, ctypes.byref(pre), 16, 16,
+                                      16, None) == dz.DZ_ERR_INVALID_ARG
+    # a null layout or output pointer is rejected before any handle lookup
+    assert lib.dz_chunk_attn_forward_lse(None, 16, 16, 16, None, 16, 16, None) == \
+        dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_chunk_attn_backward(None, 16, 16, 16, 16, 16, None, ctypes.byref(pre), 16, 16,
+                                      16, None) == dz.DZ_ERR_INVALID_ARG
 
 
 def test_python_binding_raises(lib):
