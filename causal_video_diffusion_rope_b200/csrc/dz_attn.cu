@@ -253,14 +253,6 @@ __device__ __forceinline__ void rotate_tile_row(uint8_t* tile, int r, const Rope
   }
 }
 
-// Bits j (0 <= j < 32) with lo <= j < hi.
-__device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
-  lo = max(lo, 0);
-  hi = min(hi, 32);
-  if (hi <= lo) return 0u;
-  const uint32_t up = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
-  return up & ~((1u << lo) - 1u);
-}
 
 // Scores of columns outside [la, ha) and [lb, hb) become -inf (32 columns from col0).
 __device__ __forceinline__ void mask_cols(uint32_t (&v)[32], int col0, int la, int ha, int lb,
@@ -343,14 +335,6 @@ __device__ __forceinline__ int cta_of(unsigned x, unsigned W, int G) {
   return static_cast<int>(((x + 1) * static_cast<unsigned>(G) - 1) / W);
 }
 
-// Bounded wait that ignores the abort flag (used to drain in-flight copies).
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(a, parity)) {
-    if (globaltimer() - t0 > DZ_WAIT_NS) return;
-  }
-}
 
 }  // namespace
 
@@ -494,13 +478,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       // drain: every copy this thread issued has landed before the CTA exits
       // (on the normal path all of them were consumed and these return at once)
-      if (q_loads > 0) drain_wait(&bar[B_Q_FULL], (q_loads - 1) & 1);
+      if (q_loads > 0) mbar_drain(&bar[B_Q_FULL], (q_loads - 1) & 1);
       for (int st = 0; st < KV_STAGES; ++st) {
-        if (kf_cnt[st] > 0) drain_wait(&bar[B_K_FULL + st], (kf_cnt[st] - 1) & 1);
-        if (kr_cnt[st] > 0) drain_wait(&bar[B_K_RAW + st], (kr_cnt[st] - 1) & 1);
+        if (kf_cnt[st] > 0) mbar_drain(&bar[B_K_FULL + st], (kf_cnt[st] - 1) & 1);
+        if (kr_cnt[st] > 0) mbar_drain(&bar[B_K_RAW + st], (kr_cnt[st] - 1) & 1);
       }
       for (uint32_t j = (v_iss > KV_STAGES ? v_iss - KV_STAGES : 0); j < v_iss; ++j)
-        drain_wait(&bar[B_V_FULL + j % KV_STAGES], (j / KV_STAGES) & 1);
+        mbar_drain(&bar[B_V_FULL + j % KV_STAGES], (j / KV_STAGES) & 1);
     }
   } else if (warp == WARP_MMA) {
     // ======================= tcgen05 issuer =======================
@@ -608,7 +592,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       // every issued MMA has completed before TMEM is released
       mma_commit(&bar[B_DRAIN]);
-      drain_wait(&bar[B_DRAIN], 0);
+      mbar_drain(&bar[B_DRAIN], 0);
     }
   } else {
     // ======================= rotary gate =======================

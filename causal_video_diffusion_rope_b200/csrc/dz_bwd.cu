@@ -116,21 +116,7 @@ __device__ __forceinline__ bool pair_visible(const BwdParams& p, int qt, int kt)
   return false;
 }
 
-__device__ __forceinline__ uint32_t bits_in(int lo, int hi) {
-  lo = max(lo, 0);
-  hi = min(hi, 32);
-  if (hi <= lo) return 0u;
-  const uint32_t up = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
-  return up & ~((1u << lo) - 1u);
-}
 
-__device__ __forceinline__ void bdrain(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(a, parity)) {
-    if (globaltimer() - t0 > DZ_WAIT_NS) return;
-  }
-}
 
 // Rotary position of token s (noisy teacher-forcing tokens take clean positions).
 __device__ __forceinline__ void bpos(const BwdParams& p, int s, int& t, int& h, int& w) {
@@ -245,8 +231,8 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
         tile_load(ring + BTILE, &p.tm_v, &bar[BB_FULL + st], h, kt * BT, b);
         ++it;
       }
-      bdrain(&bar[BB_FIX], 0);
-      for (uint32_t j = (it > 2 ? it - 2 : 0); j < it; ++j) bdrain(&bar[BB_FULL + (j & 1)], (j >> 1) & 1);
+      mbar_drain(&bar[BB_FIX], 0);
+      for (uint32_t j = (it > 2 ? it - 2 : 0); j < it; ++j) mbar_drain(&bar[BB_FULL + (j & 1)], (j >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -293,7 +279,7 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
       }
       mma_commit(&bar[BB_ACC]);
       mma_commit(&bar[BB_DRAIN]);
-      bdrain(&bar[BB_DRAIN], 0);
+      mbar_drain(&bar[BB_DRAIN], 0);
     }
   } else {
     const int quarter = warp & 3;
@@ -323,7 +309,7 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
         tmem_ld32(tmem + la + col + 64, dp);
         tmem_wait_ld();
         const int col0 = k0 + 64 * hf + 32 * cg;
-        const uint32_t keep = bits_in(a0 - col0, a1 - col0) | bits_in(b0 - col0, b1 - col0);
+        const uint32_t keep = range_bits(a0 - col0, a1 - col0) | range_bits(b0 - col0, b1 - col0);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -430,8 +416,8 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
         tile_load(ring + BTILE, &p.tm_do, &bar[BB_FULL + st], h, qt * BT, b);
         ++it;
       }
-      bdrain(&bar[BB_FIX], 0);
-      for (uint32_t j = (it > 2 ? it - 2 : 0); j < it; ++j) bdrain(&bar[BB_FULL + (j & 1)], (j >> 1) & 1);
+      mbar_drain(&bar[BB_FIX], 0);
+      for (uint32_t j = (it > 2 ? it - 2 : 0); j < it; ++j) mbar_drain(&bar[BB_FULL + (j & 1)], (j >> 1) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -480,7 +466,7 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
       }
       mma_commit(&bar[BB_ACC]);
       mma_commit(&bar[BB_DRAIN]);
-      bdrain(&bar[BB_DRAIN], 0);
+      mbar_drain(&bar[BB_DRAIN], 0);
     }
   } else {
     const int quarter = warp & 3;
@@ -516,7 +502,7 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
         tmem_ld32(tmem + la + col + 64, dp);
         tmem_wait_ld();
         const int qc = 64 * hf + 32 * cg;  // query column of sv[0] within the tile
-        const uint32_t keep = bits_in(a0 - q0 - qc, a1 - q0 - qc) | bits_in(b0 - q0 - qc, b1 - q0 - qc);
+        const uint32_t keep = range_bits(a0 - q0 - qc, a1 - q0 - qc) | range_bits(b0 - q0 - qc, b1 - q0 - qc);
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {

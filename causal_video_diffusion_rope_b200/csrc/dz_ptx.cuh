@@ -297,6 +297,25 @@ __device__ __forceinline__ void sts_u4(uint32_t addr, uint4 v) {
 }
 
 // ---------------------------------------------------------------- misc
+// Bounded wait that ignores the abort flag: used before exit so that copies and
+// products a role issued have finished (on the normal path they all have).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer() - t0 > DZ_WAIT_NS) return;
+  }
+}
+
+// Bits j (0 <= j < 32) with lo <= j < hi.
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi) {
+  lo = lo < 0 ? 0 : lo;
+  hi = hi > 32 ? 32 : hi;
+  if (hi <= lo) return 0u;
+  const uint32_t up = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  return up & ~((1u << lo) - 1u);
+}
+
 __device__ __forceinline__ int ld_acquire_gpu(const int* ptr) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");

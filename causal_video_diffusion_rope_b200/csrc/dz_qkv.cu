@@ -70,13 +70,6 @@ __device__ __forceinline__ void store_piece(__nv_bfloat16* dst, const uint32_t (
   for (int j = 0; j < 4; ++j) d[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
 }
 
-__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
-  const uint32_t a = smem_u32(bar);
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(a, parity)) {
-    if (globaltimer() - t0 > DZ_WAIT_NS) return;
-  }
-}
 
 }  // namespace
 
@@ -133,7 +126,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
       // every issued copy has landed before the CTA exits
       const uint32_t n_iss = it;
       for (uint32_t j = (n_iss > QSTAGES ? n_iss - QSTAGES : 0); j < n_iss; ++j)
-        drain(&bar[QB_FULL + j % QSTAGES], (j / QSTAGES) & 1);
+        mbar_drain(&bar[QB_FULL + j % QSTAGES], (j / QSTAGES) & 1);
     }
   } else if (warp == 1) {
     // ---------------- tcgen05 issuer ----------------
@@ -169,7 +162,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
         mma_commit(&bar[QB_ACC_FULL]);
       }
       mma_commit(&bar[QB_DRAIN]);
-      drain(&bar[QB_DRAIN], 0);
+      mbar_drain(&bar[QB_DRAIN], 0);
     }
   } else {
     // ---------------- epilogue: warps 2..9, one token row per thread ----------------
