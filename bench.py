@@ -627,6 +627,75 @@ def run_bwd(args, rank: int, world: int, local_rank: int, config: dict):
     print(json.dumps(line), flush=True)
 
 
+CACHE_METRIC = "KV-cache chunk replace GB/s (keys + values read and written) and % of measured HBM copy bandwidth"
+
+
+def run_cache(args, rank: int, world: int, local_rank: int, config: dict):
+    """Times dz_kvcache_replace of one chunk (every batch item's K and V rows) on the
+    workload's cache; the replaced chunk and the source set cycle, so the traffic
+    (> L2 in all) goes to HBM."""
+    import torch
+    from causal_video_diffusion_rope_b200 import dz
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    lay = w.layout
+    if not w.cache_tokens:
+        raise SystemExit("--op cache needs a workload with a KV cache (e.g. --workload 2)")
+    B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
+    n_chunks = w.cache_tokens // L
+    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B))
+    ck = torch.zeros((B, w.cache_tokens, H, D), dtype=torch.bfloat16, device=dev)
+    cv = torch.zeros_like(ck)
+    cache = dz.make_cache(ck, cv, B, w.cache_tokens, w.cache_tokens, L)
+    rng = np.random.default_rng(1000 * rank + 11)
+    srcs = [tuple(torch.from_numpy(synth.normal_bf16(rng, (B, L, H, D)).view(np.int16)).to(dev)
+                  .view(torch.bfloat16) for _ in range(2)) for _ in range(4)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def call(i):
+        k, v = srcs[i % len(srcs)]
+        dz.dz_kvcache_replace(h, cache, i % n_chunks, k, v, stream)
+
+    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    ms, clocks = time_graph(stream, call, args.steps, args.warmup, world, dev, sampler)
+    dz.dz_attn_sync_status(h, stream)
+    bytes_per = 2 * 2 * B * L * H * D * 2  # K and V, read and written
+    ms_per_step = ms / args.steps
+    gbs = bytes_per / (ms_per_step * 1e-3) / 1e9
+
+    def e2e_call(di, do):
+        dz.dz_kvcache_replace(h, cache, n_chunks - 1, di["k"], di["v"], stream)
+        with torch.cuda.stream(stream):
+            do["k_row"].copy_(ck[:, -1, 0, :8])
+
+    e2e = e2e_pipelined(dev, stream, {"k": srcs[0][0], "v": srcs[0][1]},
+                        {"k_row": torch.empty((B, 8), dtype=torch.bfloat16, device=dev)},
+                        e2e_call, max(3, min(args.steps, 200)), world)
+    e2e_ms = e2e.pop("ms")
+    e2e["value"] = round(bytes_per * e2e.pop("steps_done") * world / (e2e_ms * 1e-3) / 1e9, 2)
+    e2e["unit"] = "GB/s"
+    dz.dz_attn_destroy(h)
+    if rank != 0:
+        return
+    _, peak_hbm, peak_kind = measured_peaks()
+    line = {"metric": CACHE_METRIC, "value": round(gbs * world, 2), "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6), "us_per_call": round(ms_per_step * 1e3, 3),
+            "pct_of_hbm_peak": round(100 * gbs / peak_hbm, 2), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 (bit copy)",
+            "data": "synthetic (N(0,1) bf16 observations)",
+            "config": dict(config, op="kvcache_replace", bytes_per_step=bytes_per,
+                           l2=f"cache {2 * B * w.cache_tokens * H * D * 2 / 2**20:.0f} MiB + "
+                              f"4 source sets, replaced chunk cycling: > 126 MB L2",
+                           parallelism=f"dp{world} (independent replicas of the call)"),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak_hbm,
+                         "unit": "GB/s", "frac": round(gbs / peak_hbm, 4), "traffic": None,
+                         "peak_kind": f"{peak_kind} copy", "kernel": "kv_copy_kernel"},
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -635,9 +704,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle CPU work for the cpu_baseline field")
-    ap.add_argument("--op", default="attn", choices=["attn", "qkv", "bwd"],
+    ap.add_argument("--op", default="attn", choices=["attn", "qkv", "bwd", "cache"],
                     help="attn: the chunk-causal attention call; qkv: the fused projection; "
-                         "bwd: the backward of a prefill / teacher-forcing call")
+                         "bwd: the backward of a prefill / teacher-forcing call; "
+                         "cache: the KV-cache chunk replace")
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
                     choices=range(len(synth.WORKLOADS)),
                     help="workload index (default: the single-layer inference step)")
@@ -657,7 +727,7 @@ def main():
               "rope": "3d t/h/w 22/21/21 base 1e4; q and the chunk's k rotated once per call",
               "flop_per_step": step_flops(w)}
 
-    if args.op in ("qkv", "bwd"):
+    if args.op in ("qkv", "bwd", "cache"):
         if args.impl == "reference":
             if rank == 0:
                 print(json.dumps({"impl": "reference", "unavailable": "the reference arm times "
@@ -667,7 +737,8 @@ def main():
         if world > 1:
             import datetime
             dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        (run_qkv if args.op == "qkv" else run_bwd)(args, rank, world, local_rank, config)
+        {"qkv": run_qkv, "bwd": run_bwd, "cache": run_cache}[args.op](args, rank, world,
+                                                                     local_rank, config)
         if world > 1:
             dist.barrier()
             dist.destroy_process_group()
