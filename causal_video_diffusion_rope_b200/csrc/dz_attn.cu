@@ -29,9 +29,12 @@
 // Work split (stream-K): unit = (batch, head, group of 256 query rows); its
 // key tiles are the tiles any of its rows can see (fully masked tiles are never
 // loaded).  All units' tiles are laid end to end and cut into one contiguous
-// range per CTA.  A unit that one CTA covers entirely writes bf16 output
-// directly; otherwise every piece writes fp32 partial (O, m, l) to the
-// workspace and the last piece to finish (atomic counter) merges them.
+// range per CTA (one CTA per unit when that is no slower).  A unit that one
+// CTA covers entirely writes bf16 output directly; otherwise each piece counts
+// its arrival on the unit's counter, every piece but the last to arrive
+// publishes fp32 partial (O, m, l) to the workspace, and the last one merges
+// them into its own O in TMEM.  With the call's q and own k rotated once into a
+// workspace beforehand (or given rotated), the rotary gate only passes tiles on.
 #include "dz_internal.cuh"
 #include "dz_ptx.cuh"
 
