@@ -86,7 +86,7 @@ class Workload:
         return 128
 
 
-# The five workloads; index i is "config i" in tests and the benchmark.
+# The workloads; index i is "workload i" in tests and the benchmark.
 WORKLOADS = [
     Workload(
         "tiny_prefill_b1_h2_3x36", heads=2,
