@@ -100,3 +100,35 @@ def test_binding_has_same_names_as_header():
     declared = _declared_functions()
     for name in declared:
         assert hasattr(dz, name), f"binding lacks {name}"
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """Size and field offsets of the public structs as a C compiler lays them out from
+    include/dz.h, against the binding's ctypes definitions."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    structs = {"dz_attn_desc": dz.dz_attn_desc, "dz_chunk_layout": dz.dz_chunk_layout,
+               "dz_kvcache": dz.dz_kvcache}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "dz.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} size %zu\\n", sizeof({name}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{name} {field} %zu\\n", offsetof({name}, {field}));')
+    lines += ['  printf("DZ_MODE_ROTATED %d\\n", DZ_MODE_ROTATED);', "  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n"):
+        if line:
+            *key, value = line.split()
+            got[" ".join(key)] = int(value)
+    for name, cls in structs.items():
+        assert got[f"{name} size"] == ctypes.sizeof(cls), name
+        for field, _ in cls._fields_:
+            assert got[f"{name} {field}"] == getattr(cls, field).offset, (name, field)
+    assert got["DZ_MODE_ROTATED"] == dz.DZ_MODE_ROTATED
