@@ -14,7 +14,7 @@ import torch
 
 from causal_video_diffusion_rope_b200 import dz, synth
 from causal_video_diffusion_rope_b200.synth import MODE_DECODE, MODE_PREFILL
-from gpu_util import Handle, assert_close, to_bits, to_dev, to_f64
+from gpu_util import Handle, to_bits, to_dev, to_f64
 from oracle import dz_oracle as O
 
 pytestmark = pytest.mark.gpu

@@ -10,7 +10,6 @@ collected last so that a failure here does not hide the other tests.
 """
 import ctypes
 
-import numpy as np
 import pytest
 import torch
 
