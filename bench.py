@@ -788,7 +788,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     cpu = None
-    if rank == 0 and args.cpu_budget > 0:
+    if rank == 0 and world == 1 and args.cpu_budget > 0:
         # the oracle, timed on this host's cores before the GPU work starts
         r, heads_done, dt = oracle_full_call_rate(w, args.cpu_budget)
         cpu = {"value": round(r, 6), "unit": "TFLOP/s", "cores": blas_threads(),
