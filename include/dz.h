@@ -172,7 +172,8 @@ dz_status dz_rope3d(dz_attn_t handle, const void* x, void* y, int32_t B, int32_t
                     const dz_chunk_layout* layout, int32_t first_chunk, void* stream);
 
 /* Chunk-causal attention: out = softmax(R q (R k)^T / sqrt(128), chunk mask) v
- * per batch item and head, for the mode in `layout` (see dz_mode).
+ * per batch item and head, for the mode in `layout` (see dz_mode; with
+ * DZ_MODE_ROTATED or-ed in, q and k are taken as already rotated).
  *   q    bf16 [B][Sq][H][128]; Sq = L (DECODE), 2*N*L (TEACHER_FORCING),
  *        N*L (PREFILL, CROSS).
  *   k, v bf16 [B][Sk][H][128]; Sk = Sq, or kv_len for CROSS.
