@@ -12,8 +12,16 @@ online softmax, PV and the split-KV combine.
 Prints ONE JSON line on rank 0.  Timing: K calls replayed from CUDA graphs
 that cycle through enough distinct input sets to exceed the 126 MB L2, timed
 with CUDA events on the launching stream between barriers + synchronize, max
-over ranks.  ``--impl reference`` times the CPU fp64 oracle instead (bounded
-samples of the same workload per step).
+over ranks.  At N=1 the line also carries a `workloads` block with the other
+full-size workloads (CFG decode with its cache replace, teacher forcing, long
+cache + cross-attention, three-view decode) timed the same way.
+
+With --gpus N and no launcher environment (WORLD_SIZE unset) the script starts
+N rank processes itself, one per GPU.  Ranks share no data: on a workload whose
+batch equals N (the CFG branches), rank r runs branch r's batch-1 calls against
+its own half of the cache (the two-GPU CFG split); otherwise every rank runs
+its own replica of the call.  ``--impl reference`` times the CPU fp64 oracle
+instead (bounded samples of the same workload per step).
 """
 from __future__ import annotations
 
@@ -23,6 +31,7 @@ import json
 import math
 import os
 import re
+import socket
 import subprocess
 import sys
 import time
@@ -37,7 +46,9 @@ from causal_video_diffusion_rope_b200 import synth  # noqa: E402
 METRIC = ("chunk-causal attn TFLOP/s and % of B200 BF16 peak; "
           "µs per DiT-layer attention call")
 DEFAULT_WORKLOAD = 1  # single DiT-layer inference step
+EXTRA_WORKLOADS = (2, 3, 4, 5)
 L2_BYTES = 126 * 1024 * 1024
+SPEC_BF16_TFLOPS = 2250.0  # B200 dense bf16, the figure the throughput aim is stated against
 KERNEL_SOURCES = ["causal_video_diffusion_rope_b200/csrc/dz_attn.cu",
                   "causal_video_diffusion_rope_b200/csrc/dz_internal.cuh",
                   "causal_video_diffusion_rope_b200/csrc/dz_ptx.cuh"]
@@ -59,14 +70,21 @@ def visible_pairs(w: synth.Workload) -> int:
     return clean + noisy
 
 
+def self_flops(w: synth.Workload) -> float:
+    """Algorithmic FLOPs of the self-attention call: 4 * head_dim per visible (query, key)
+    pair per head per batch item."""
+    return 4.0 * w.head_dim * visible_pairs(w) * w.heads * w.layout.batch
+
+
+def cross_flops(w: synth.Workload) -> float:
+    """Algorithmic FLOPs of the cross-attention call (every condition key visible)."""
+    return 4.0 * w.head_dim * w.layout.chunk_len * w.cross_kv_len * w.heads * w.layout.batch
+
+
 def step_flops(w: synth.Workload) -> float:
-    """Algorithmic FLOPs of one step: 4 * head_dim per visible (query, key) pair per head per
-    batch item, for the self-attention call plus, in the long-cache workload, the
-    cross-attention call (every key visible)."""
-    f = 4.0 * w.head_dim * visible_pairs(w) * w.heads * w.layout.batch
-    if w.cross_kv_len:
-        f += 4.0 * w.head_dim * w.layout.chunk_len * w.cross_kv_len * w.heads * w.layout.batch
-    return f
+    """Algorithmic FLOPs of one step: the self-attention call plus, in the long-cache
+    workload, the cross-attention call."""
+    return self_flops(w) + (cross_flops(w) if w.cross_kv_len else 0.0)
 
 
 def step_bytes(w: synth.Workload) -> float:
@@ -80,10 +98,11 @@ def step_bytes(w: synth.Workload) -> float:
     return row * n
 
 
-def launches_per_step(w: synth.Workload) -> int:
-    """Kernels of this library one step launches: the once-per-call rotation of q and k and
-    the attention kernel, plus the cross-attention kernel in the long-cache workload."""
-    return 2 + (1 if w.cross_kv_len else 0)
+def launches_per_step(w: synth.Workload, rotation_pass: bool) -> int:
+    """Kernels of this library one step launches: the attention kernel (plus the
+    once-per-call rotation of q and k when it runs as its own pass), plus the
+    cross-attention kernel in the long-cache workload."""
+    return 1 + (1 if rotation_pass else 0) + (1 if w.cross_kv_len else 0)
 
 
 def sources_hash() -> str:
@@ -108,10 +127,11 @@ def measured_peaks():
     return 1590.0, 6650.0, "fallback"
 
 
-def ncu_traffic():
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary,
-    or None if it was taken on different kernel sources."""
-    path = os.path.join(ROOT, "profiles", "attn_decode_b1_h40_q464_cache4.json")
+def ncu_traffic(workload_name: str):
+    """Per-launch DRAM bytes of the attention kernel on a workload from the committed ncu
+    summary (profiles/attn_<workload>.json), or None if there is none or it was taken on
+    different kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"attn_{workload_name}.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
@@ -121,22 +141,57 @@ def ncu_traffic():
     return d.get("dram_bytes_per_launch")
 
 
+def cpu_info():
+    """CPU model name and the cores this process may run on."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        cores = len(os.sched_getaffinity(0))
+    except AttributeError:
+        cores = os.cpu_count()
+    return model, cores
+
+
+def gpu_id(local_rank: int) -> str:
+    """nvidia-smi --id of this rank's GPU: its UUID (the leased GPU, whatever
+    CUDA_VISIBLE_DEVICES maps it to), else the CUDA_VISIBLE_DEVICES entry, else the index."""
+    try:
+        import torch
+        u = str(torch.cuda.get_device_properties(local_rank).uuid)
+        if u:
+            return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        pass
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        entries = [e.strip() for e in vis.split(",") if e.strip()]
+        if local_rank < len(entries):
+            return entries[local_rank]
+    return str(local_rank)
+
+
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling in the background."""
+    """nvidia-smi clock / throttle sampling of one GPU in the background."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, gpu: str):
+        self.gpu = gpu
         self.proc = None
-        self.t_on = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
@@ -144,7 +199,8 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "gpu": self.gpu}
         time.sleep(0.25)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
@@ -163,7 +219,7 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "gpu": self.gpu}
 
 
 # ----------------------------------------------------------------------------------- CPU legs
@@ -203,6 +259,16 @@ def blas_threads() -> int:
         return 1
 
 
+def cpu_baseline_fields(value: float, sample: str) -> dict:
+    """cpu_baseline object: `cores` = the threads the oracle's matrix products ran on
+    (the BLAS pool, bounded by this process's CPU affinity), with the affinity core
+    count and the CPU model beside it."""
+    model, avail = cpu_info()
+    used = min(blas_threads(), avail) if avail else blas_threads()
+    return {"value": round(value, 6), "unit": "TFLOP/s", "cores": used,
+            "cores_available": avail, "cpu_model": model, "kind": "oracle", "sample": sample}
+
+
 def oracle_full_call_rate(w: synth.Workload, budget_s: float):
     """The oracle computing whole calls of ``w`` (all heads) for about ``budget_s``."""
     from oracle import dz_oracle as O
@@ -222,12 +288,49 @@ def oracle_full_call_rate(w: synth.Workload, budget_s: float):
         heads_done += 4
         n += 1
     dt = time.perf_counter() - t0
-    self_flops = 4.0 * w.head_dim * visible_pairs(w) * w.layout.batch
-    flops = self_flops * heads_done
+    flops = visible_pairs(w) * 4.0 * w.head_dim * w.layout.batch * heads_done
     return flops / dt / 1e12, heads_done, dt
 
 
 # ----------------------------------------------------------------------------------- ranks
+
+def free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_ranks(n: int, target, *args) -> None:
+    """Run ``target(*args)`` in ``n`` fresh processes (spawn), one per GPU rank, with the
+    launcher environment a rank expects (RANK, LOCAL_RANK, WORLD_SIZE, MASTER_ADDR,
+    MASTER_PORT); raises if any rank fails."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    port = free_port()
+    procs = [ctx.Process(target=_rank_entry, args=(r, n, port, target, args)) for r in range(n)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join()
+    bad = [(r, p.exitcode) for r, p in enumerate(procs) if p.exitcode != 0]
+    if bad:
+        raise RuntimeError(f"rank processes failed: {bad}")
+
+
+def _rank_entry(rank: int, world: int, port: int, target, args) -> None:
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    target(*args)
+
+
+def rank_work(w: synth.Workload, rank: int, world: int):
+    """What one rank runs of workload ``w``: ("cfg", r) -- branch r of a batch whose items
+    are the CFG branches, one rank per branch (world == batch > 1) -- or ("replica", None),
+    its own copy of the whole call."""
+    if world > 1 and w.layout.batch == world:
+        return "cfg", rank
+    return "replica", None
+
 
 def max_over_ranks(ms: float, world: int, device) -> float:
     """The slowest rank's time: every rank's elapsed milliseconds reduced with MAX."""
@@ -241,8 +344,8 @@ def max_over_ranks(ms: float, world: int, device) -> float:
 
 
 def job_throughput(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
-    """Whole-job TFLOP/s: every rank runs `steps` independent calls (weak scaling);
-    the job takes as long as its slowest rank."""
+    """Whole-job TFLOP/s: every rank runs `steps` calls of `flops_per_step` each; the job
+    takes as long as its slowest rank."""
     return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
 
 
@@ -313,139 +416,6 @@ def e2e_pipelined(dev, stream, dev_inputs: dict, dev_outputs: dict, call, n_step
             "ms_per_step": round(ms / n_steps, 4), "steps": n_steps}
 
 
-# ----------------------------------------------------------------------------------- GPU leg
-
-def run_gpu(args, rank: int, world: int, local_rank: int):
-    import torch
-    import torch.distributed as dist
-    from causal_video_diffusion_rope_b200 import dz
-
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    w = synth.WORKLOADS[args.workload]
-    lay = w.layout
-    B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
-    per_set = step_bytes(w)
-    n_sets = max(2, int(math.ceil(3 * L2_BYTES / per_set)))
-    # q and the chunk's own k are rotated once per call (prerotate_tokens) before the
-    # attention kernel; cache keys are stored rotated
-    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len,
-                                       prerotate_tokens=lay.q_len))
-    dl = dz.layout_from(lay)
-    dlx = dz.layout_from(synth.cross_layout(w)) if w.cross_kv_len else None
-    sets = []
-    for i in range(n_sets):
-        inp = synth.make_inputs(w, 1000 * rank + i)
-        s = {k: torch.from_numpy(inp[k].view(np.int16)).to(dev).view(torch.bfloat16)
-             for k in ("q", "k", "v", "cache_k", "cache_v", "q_x", "k_x", "v_x") if k in inp}
-        s["out"] = torch.empty((B, lay.q_len, H, D), dtype=torch.bfloat16, device=dev)
-        s["cache"] = (dz.make_cache(s["cache_k"], s["cache_v"], B, w.cache_tokens,
-                                    w.cache_tokens, L) if "cache_k" in s else None)
-        if w.cross_kv_len:
-            s["out_x"] = torch.empty((B, L, H, D), dtype=torch.bfloat16, device=dev)
-        sets.append(s)
-    stream = torch.cuda.Stream(device=dev)
-
-    def call(i):
-        s = sets[i % n_sets]
-        dz.dz_chunk_attn_forward(h, s["q"], s["k"], s["v"], s["cache"], dl, s["out"], stream)
-        if dlx is not None:
-            dz.dz_chunk_attn_forward(h, s["q_x"], s["k_x"], s["v_x"], None, dlx, s["out_x"],
-                                     stream)
-
-    # warm-up outside any graph
-    with torch.cuda.stream(stream):
-        for i in range(max(args.warmup, 3)):
-            call(i)
-    stream.synchronize()
-    dz.dz_attn_sync_status(h, stream)
-
-    # graphs of g calls cycling through the input sets
-    g = n_sets * max(1, 240 // n_sets)
-    graphs = {}
-
-    def graph_of(n):
-        if n not in graphs:
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=stream):
-                for i in range(n):
-                    call(i)
-            graphs[n] = gr
-        return graphs[n]
-
-    full, rem = divmod(args.steps, g)
-    if full:
-        graph_of(g)
-    if rem:
-        graph_of(rem)
-    # warm the graphs once
-    with torch.cuda.stream(stream):
-        if full:
-            graphs[g].replay()
-        if rem:
-            graphs[rem].replay()
-    stream.synchronize()
-
-    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
-    sampler.start()
-    time.sleep(0.3)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(full):
-            graphs[g].replay()
-        if rem:
-            graphs[rem].replay()
-        e1.record(stream)
-    stream.synchronize()
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop()
-    ms = e0.elapsed_time(e1)
-    dz.dz_attn_sync_status(h, stream)
-    ms = max_over_ranks(ms, world, dev)
-    ms_per_step = ms / args.steps
-    flops = step_flops(w)
-    tflops_total = job_throughput(flops, args.steps, world, ms)
-
-    # ---- end to end: host buffers in, result out, through the same C-ABI calls
-    s0 = sets[0]
-    in_keys = [k for k in ("q", "k", "v", "q_x", "k_x", "v_x") if k in s0]
-    out_keys = [k for k in ("out", "out_x") if k in s0]
-
-    def e2e_call(di, do):
-        dz.dz_chunk_attn_forward(h, di["q"], di["k"], di["v"], s0["cache"], dl, do["out"], stream)
-        if dlx is not None:
-            dz.dz_chunk_attn_forward(h, di["q_x"], di["k_x"], di["v_x"], None, dlx,
-                                     do["out_x"], stream)
-
-    e2e = e2e_pipelined(dev, stream, {k: s0[k] for k in in_keys}, {k: s0[k] for k in out_keys},
-                        e2e_call, max(3, min(args.steps, 200)), world)
-    dz.dz_attn_sync_status(h, stream)
-    e2e["value"] = round(job_throughput(flops, e2e.pop("steps_done"), world, e2e.pop("ms")), 3)
-
-    for gr in graphs.values():
-        del gr
-    graphs.clear()
-    dz.dz_attn_destroy(h)
-    return ms_per_step, tflops_total, clocks, e2e
-
-
-QKV_METRIC = ("fused QKV projection + 3D RoPE TFLOP/s and % of B200 BF16 peak; "
-              "\u00b5s per DiT-layer projection of one chunk")
-D_MODEL = 5120  # hidden size of the 14B DiT
-
-
-def qkv_flops(w) -> float:
-    lay = w.layout
-    return 2.0 * lay.batch * lay.chunk_len * D_MODEL * 3 * w.heads * w.head_dim
-
-
 def time_graph(stream, call, steps: int, warmup: int, world: int, dev, sampler=None):
     """Device time (ms, max over ranks) of `steps` calls replayed from CUDA graphs of up to
     240 calls, after `warmup` plain calls and one replay of each graph."""
@@ -484,10 +454,186 @@ def time_graph(stream, call, steps: int, warmup: int, world: int, dev, sampler=N
             graphs[rem].replay()
         e1.record(stream)
     stream.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
     clocks = sampler.stop() if sampler else None
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     graphs.clear()
     return ms, clocks
+
+
+# ----------------------------------------------------------------------------------- GPU legs
+
+class AttnSetup:
+    """Handle, input sets and layouts of one workload's attention calls on this rank.
+
+    Input sets cycle so that one pass over them exceeds the L2 (every call reads its
+    q, k, v and cache from HBM).  ``branch`` selects one batch item of the workload
+    (a CFG branch, with its own half of the cache); the seeds do not depend on the
+    rank in that case, so the ranks together run exactly the batch-2 call."""
+
+    def __init__(self, w: synth.Workload, dev, seed_base: int, rotation_pass: bool,
+                 branch=None, max_sets=None):
+        import torch
+        from causal_video_diffusion_rope_b200 import dz
+        self.dz = dz
+        self.w_full = w
+        self.w = w if branch is None else synth.branch_inputs(w, {}, branch)[0]
+        lay = self.w.layout
+        B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
+        self.n_sets = max(2, int(math.ceil(3 * L2_BYTES / step_bytes(self.w))))
+        if max_sets:
+            self.n_sets = min(self.n_sets, max_sets)
+        self.h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len,
+                                                prerotate_tokens=lay.q_len if rotation_pass else 0))
+        self.dl = dz.layout_from(lay)
+        self.dlx = dz.layout_from(synth.cross_layout(self.w)) if w.cross_kv_len else None
+        self.sets = []
+        for i in range(self.n_sets):
+            inp = synth.make_inputs(w, seed_base + i)
+            if branch is not None:
+                inp = synth.branch_inputs(w, inp, branch)[1]
+            s = {k: torch.from_numpy(np.ascontiguousarray(inp[k]).view(np.int16)).to(dev)
+                 .view(torch.bfloat16)
+                 for k in ("q", "k", "v", "cache_k", "cache_v", "q_x", "k_x", "v_x") if k in inp}
+            s["out"] = torch.empty((B, lay.q_len, H, D), dtype=torch.bfloat16, device=dev)
+            s["cache"] = (dz.make_cache(s["cache_k"], s["cache_v"], B, self.w.cache_tokens,
+                                        self.w.cache_tokens, L) if "cache_k" in s else None)
+            if w.cross_kv_len:
+                s["out_x"] = torch.empty((B, L, H, D), dtype=torch.bfloat16, device=dev)
+            self.sets.append(s)
+
+    def call(self, i, stream, part="step"):
+        """One step on input set i: the self-attention call, plus the cross-attention call
+        of the long-cache workload (part: "step" both, "self" or "cross" one of them)."""
+        s = self.sets[i % self.n_sets]
+        if part in ("step", "self"):
+            self.dz.dz_chunk_attn_forward(self.h, s["q"], s["k"], s["v"], s["cache"], self.dl,
+                                          s["out"], stream)
+        if self.dlx is not None and part in ("step", "cross"):
+            self.dz.dz_chunk_attn_forward(self.h, s["q_x"], s["k_x"], s["v_x"], None, self.dlx,
+                                          s["out_x"], stream)
+
+    def close(self):
+        self.dz.dz_attn_sync_status(self.h)
+        self.dz.dz_attn_destroy(self.h)
+        self.sets.clear()
+
+
+def extra_workload_block(wl: int, dev, stream, steps: int, peak_tf: float, peak_hbm: float):
+    """Timing of one more full-size workload (N=1), the headline's discipline: graphs of
+    calls cycling input sets above L2, CUDA events on the launching stream."""
+    import torch
+    w = synth.WORKLOADS[wl]
+    st = AttnSetup(w, dev, 2000 + 100 * wl, rotation_pass=False, max_sets=3)
+    n = max(20, min(steps, 240))
+    res = {"workload": w.name, "mode": synth.MODE_NAMES[w.layout.mode],
+           "batch": w.layout.batch, "q_tokens": w.layout.q_len,
+           "keys": w.cache_tokens + w.layout.self_kv_len, "calls": n,
+           "l2": f"{st.n_sets} input sets of {step_bytes(w) / 2**20:.0f} MiB cycle"}
+    ms, _ = time_graph(stream, lambda i: st.call(i, stream), n, 3, 1, dev)
+    us = 1e3 * ms / n
+    tf = step_flops(w) / (us * 1e-6) / 1e12
+    res.update(us_per_call=round(us, 3), tflops=round(tf, 2), frac=round(tf / peak_tf, 4),
+               frac_of_spec=round(tf / SPEC_BF16_TFLOPS, 4), flop_per_call=step_flops(w),
+               traffic=ncu_traffic(w.name))
+    if w.cross_kv_len:
+        for part, fl in (("self", self_flops(w)), ("cross", cross_flops(w))):
+            ms, _ = time_graph(stream, lambda i, part=part: st.call(i, stream, part), n, 3, 1, dev)
+            pus = 1e3 * ms / n
+            ptf = fl / (pus * 1e-6) / 1e12
+            res[part] = {"us_per_call": round(pus, 3), "tflops": round(ptf, 2),
+                         "frac": round(ptf / peak_tf, 4), "flop_per_call": fl}
+    if w.denoise_steps > 1 and st.sets[0]["cache"] is not None:
+        # the request boundary: the observed chunk replaces the last cached chunk
+        dz = st.dz
+        lay = w.layout
+        L = lay.chunk_len
+        srcs = [(torch.randn((lay.batch, L, w.heads, w.head_dim), device=dev).to(torch.bfloat16),
+                 torch.randn((lay.batch, L, w.heads, w.head_dim), device=dev).to(torch.bfloat16))
+                for _ in range(4)]
+        last = w.cache_tokens // L - 1
+
+        def rep(i):
+            s = st.sets[i % st.n_sets]
+            k, v = srcs[i % len(srcs)]
+            dz.dz_kvcache_replace(st.h, s["cache"], last, k, v, stream)
+
+        ms, _ = time_graph(stream, rep, n, 3, 1, dev)
+        rus = 1e3 * ms / n
+        moved = 2 * 2 * lay.batch * L * w.heads * w.head_dim * 2  # K and V, read and written
+        res["replace"] = {"us_per_call": round(rus, 3), "bytes": moved,
+                          "gbs": round(moved / (rus * 1e-6) / 1e9, 1),
+                          "frac_of_hbm": round(moved / (rus * 1e-6) / 1e9 / peak_hbm, 4)}
+    st.close()
+    del st
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_attention(args, rank: int, world: int, local_rank: int):
+    """The headline: K steps of the attention call on this rank, timed with CUDA events
+    (max over ranks); then the end-to-end leg through the same C-ABI call with host
+    buffers.  Returns (ms_per_step, job TFLOP/s, clocks, e2e, what this rank ran)."""
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    kind, branch = rank_work(w, rank, world)
+    seed_base = 1000 if kind == "cfg" else 1000 * rank
+    rotation_pass = args.rotation == "pass"
+    st = AttnSetup(w, dev, seed_base, rotation_pass, branch=branch)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            st.call(i, stream)
+    stream.synchronize()
+    st.dz.dz_attn_sync_status(st.h, stream)
+    sampler = ClockSampler(gpu_id(local_rank))
+    ms, clocks = time_graph(stream, lambda i: st.call(i, stream), args.steps, 0, world, dev,
+                            sampler)
+    st.dz.dz_attn_sync_status(st.h, stream)
+    ms_per_step = ms / args.steps
+    flops_rank = step_flops(st.w)  # this rank's share of one step
+    tflops_total = job_throughput(flops_rank, args.steps, world, ms)
+
+    # ---- end to end: host buffers in, result out, through the same C-ABI calls
+    s0 = st.sets[0]
+    in_keys = [k for k in ("q", "k", "v", "q_x", "k_x", "v_x") if k in s0]
+    out_keys = [k for k in ("out", "out_x") if k in s0]
+
+    def e2e_call(di, do):
+        st.dz.dz_chunk_attn_forward(st.h, di["q"], di["k"], di["v"], s0["cache"], st.dl,
+                                    do["out"], stream)
+        if st.dlx is not None:
+            st.dz.dz_chunk_attn_forward(st.h, di["q_x"], di["k_x"], di["v_x"], None, st.dlx,
+                                        do["out_x"], stream)
+
+    e2e = e2e_pipelined(dev, stream, {k: s0[k] for k in in_keys}, {k: s0[k] for k in out_keys},
+                        e2e_call, max(3, min(args.steps, 200)), world)
+    st.dz.dz_attn_sync_status(st.h, stream)
+    e2e["value"] = round(job_throughput(flops_rank, e2e.pop("steps_done"), world, e2e.pop("ms")), 3)
+    ran = {"kind": kind, "branch": branch, "batch_per_rank": st.w.layout.batch,
+           "n_sets": st.n_sets, "set_bytes": step_bytes(st.w)}
+    st.close()
+    extra = None
+    if world == 1 and args.extra:
+        peak_tf, peak_hbm, _ = measured_peaks()
+        extra = [extra_workload_block(x, dev, stream, args.steps, peak_tf, peak_hbm)
+                 for x in EXTRA_WORKLOADS if x != args.workload]
+    return ms_per_step, tflops_total, clocks, e2e, ran, extra
+
+
+QKV_METRIC = ("fused QKV projection + 3D RoPE TFLOP/s and % of B200 BF16 peak; "
+              "\u00b5s per DiT-layer projection of one chunk")
+D_MODEL = 5120  # hidden size of the 14B DiT
+
+
+def qkv_flops(w) -> float:
+    lay = w.layout
+    return 2.0 * lay.batch * lay.chunk_len * D_MODEL * 3 * w.heads * w.head_dim
 
 
 def run_qkv(args, rank: int, world: int, local_rank: int, config: dict):
@@ -515,7 +661,7 @@ def run_qkv(args, rank: int, world: int, local_rank: int, config: dict):
     def call(i):
         dz.dz_qkv_rope(h, xs[i % 2], W, B, S, D_MODEL, dl, first, q, k, v, None, stream)
 
-    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    sampler = ClockSampler(gpu_id(local_rank))
     ms, clocks = time_graph(stream, call, args.steps, args.warmup, world, dev, sampler)
     dz.dz_attn_sync_status(h, stream)
     ms_per_step = ms / args.steps
@@ -597,7 +743,7 @@ def run_bwd(args, rank: int, world: int, local_rank: int, config: dict):
     def call(i):
         dz.dz_chunk_attn_backward(h, q, k, v, out, dout, lse, dl, dq, dk, dv, stream)
 
-    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    sampler = ClockSampler(gpu_id(local_rank))
     ms, clocks = time_graph(stream, call, args.steps, args.warmup, world, dev, sampler)
     dz.dz_attn_sync_status(h, stream)
     ms_per_step = ms / args.steps
@@ -663,7 +809,7 @@ def run_cache(args, rank: int, world: int, local_rank: int, config: dict):
         k, v = srcs[i % len(srcs)]
         dz.dz_kvcache_replace(h, cache, i % n_chunks, k, v, stream)
 
-    sampler = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    sampler = ClockSampler(gpu_id(local_rank))
     ms, clocks = time_graph(stream, call, args.steps, args.warmup, world, dev, sampler)
     dz.dz_attn_sync_status(h, stream)
     bytes_per = 2 * 2 * B * L * H * D * 2  # K and V, read and written
@@ -702,7 +848,35 @@ def run_cache(args, rank: int, world: int, local_rank: int, config: dict):
     print(json.dumps(line), flush=True)
 
 
-def main():
+def reference_line(args, w, config) -> dict:
+    """The reference arm: the CPU fp64 oracle as it stands, on bounded samples of the
+    same workload (one sampled query row per step)."""
+    budget = 150.0 / (args.steps + args.warmup)
+    rows_per_step = 1
+    rate = []
+    t_all = time.perf_counter()
+    inp = synth.make_inputs(w, 0)
+    rng = np.random.default_rng(0)
+    for i in range(args.warmup + args.steps):
+        r, calls, dt = oracle_rate(w, inp, rng, budget, rows_per_step)
+        if i >= args.warmup:
+            rate.append((r, dt))
+    elapsed = sum(dt for _, dt in rate)
+    value = float(np.mean([r for r, _ in rate]))
+    sample = (f"{rows_per_step} query row(s) of the call per step, "
+              f"~{budget * 1e3:.1f} ms of oracle work per step")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6),
+            "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / max(1, len(rate)), 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": dict(config, l2="n/a (CPU)"),
+            "cpu_baseline": cpu_baseline_fields(value, sample),
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": round(time.perf_counter() - t_all, 1)}
+
+
+def parse_args(argv):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=48000)
@@ -717,10 +891,20 @@ def main():
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
                     choices=range(len(synth.WORKLOADS)),
                     help="workload index (default: the single-layer inference step)")
-    args = ap.parse_args()
+    ap.add_argument("--rotation", default="kernel", choices=["kernel", "pass"],
+                    help="kernel: q and the chunk's k rotated as the attention kernel loads "
+                         "them; pass: rotated once per call by a separate kernel first")
+    ap.add_argument("--no-extra", dest="extra", action="store_false",
+                    help="skip the other workloads' block of the headline line")
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
+    return args
 
+
+def rank_main(argv) -> None:
+    """One rank's work (rank, world and local rank come from the launcher environment)."""
+    args = parse_args(argv)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
@@ -730,97 +914,85 @@ def main():
               "keys": w.cache_tokens + w.layout.self_kv_len, "cache_tokens": w.cache_tokens,
               "mode": synth.MODE_NAMES[w.layout.mode],
               "cross_keys": w.cross_kv_len,
-              "rope": "3d t/h/w 22/21/21 base 1e4; q and the chunk's k rotated once per call",
+              "rope": ("3d t/h/w 22/21/21 base 1e4; q and the chunk's k rotated " +
+                       ("as the attention kernel loads them" if args.rotation == "kernel"
+                        else "once per call by a separate kernel")),
               "flop_per_step": step_flops(w)}
 
-    if args.op in ("qkv", "bwd", "cache"):
-        if args.impl == "reference":
-            if rank == 0:
+    if args.impl == "reference":
+        # rank 0 alone runs the oracle; other ranks exit without work
+        if rank == 0:
+            if args.op != "attn":
                 print(json.dumps({"impl": "reference", "unavailable": "the reference arm times "
                                   "the attention call (--op attn) only"}), flush=True)
-            return
-        import torch.distributed as dist
-        if world > 1:
-            import datetime
-            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        {"qkv": run_qkv, "bwd": run_bwd, "cache": run_cache}[args.op](args, rank, world,
-                                                                     local_rank, config)
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
+            else:
+                print(json.dumps(reference_line(args, w, config)), flush=True)
         return
 
-    if args.impl == "reference":
-        if rank != 0:
-            return
-        budget = 150.0 / (args.steps + args.warmup)
-        # each step: the oracle on a bounded sample of query rows of the same call
-        rows_per_step = 1
-        rate = []
-        t_all = time.perf_counter()
-        inp = synth.make_inputs(w, 0)
-        rng = np.random.default_rng(0)
-        for i in range(args.warmup + args.steps):
-            r, calls, dt = oracle_rate(w, inp, rng, budget, rows_per_step)
-            if i >= args.warmup:
-                rate.append((r, dt))
-        elapsed = sum(dt for _, dt in rate)
-        value = float(np.mean([r for r, _ in rate]))
-        cores = blas_threads()
-        line = {"impl": "reference", "metric": METRIC, "value": round(value, 6),
-                "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": round(1e3 * elapsed / max(1, len(rate)), 3),
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                "data": "synthetic", "config": dict(config, l2="n/a (CPU)"),
-                "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cores,
-                                 "kind": "oracle",
-                                 "sample": f"{rows_per_step} query row(s) of the call per step, "
-                                           f"~{budget * 1e3:.1f} ms of oracle work per step"},
-                "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0},
-                "wall_s": round(time.perf_counter() - t_all, 1)}
-        print(json.dumps(line), flush=True)
-        return
-
-    import torch
     import torch.distributed as dist
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    cpu = None
-    if rank == 0 and world == 1 and args.cpu_budget > 0:
-        # the oracle, timed on this host's cores before the GPU work starts
-        r, heads_done, dt = oracle_full_call_rate(w, args.cpu_budget)
-        cpu = {"value": round(r, 6), "unit": "TFLOP/s", "cores": blas_threads(),
-               "kind": "oracle",
-               "sample": f"{heads_done} of {w.heads} heads of the call (4-head slices), "
-                         f"{dt:.1f} s of fp64 oracle work"}
-    ms_per_step, tflops, clocks, e2e = run_gpu(args, rank, world, local_rank)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    try:
+        if args.op in ("qkv", "bwd", "cache"):
+            {"qkv": run_qkv, "bwd": run_bwd, "cache": run_cache}[args.op](args, rank, world,
+                                                                         local_rank, config)
+            return
+        cpu = None
+        if rank == 0 and world == 1 and args.cpu_budget > 0:
+            # the oracle, timed on this host's cores before the GPU work starts
+            r, heads_done, dt = oracle_full_call_rate(w, args.cpu_budget)
+            cpu = cpu_baseline_fields(r, f"{heads_done} of {w.heads} heads of the call "
+                                         f"(4-head slices), {dt:.1f} s of fp64 oracle work")
+        ms_per_step, tflops, clocks, e2e, ran, extra = run_attention(args, rank, world,
+                                                                     local_rank)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
     if rank != 0:
         return
     peak_tf, peak_hbm, peak_kind = measured_peaks()
-    per_gpu_tf = step_flops(w) / (ms_per_step * 1e-3) / 1e12
+    # this rank's share of a step: the whole call (replicas) or one CFG branch of it
+    w_rank = synth.branch_inputs(w, {}, 0)[0] if ran["kind"] == "cfg" else w
+    per_gpu_tf = step_flops(w_rank) / (ms_per_step * 1e-3) / 1e12
+    rotation_pass = args.rotation == "pass"
     roof = {"bound": "tensor", "achieved": round(per_gpu_tf, 2), "peak": peak_tf,
             "unit": "TFLOP/s", "frac": round(per_gpu_tf / peak_tf, 4),
-            "traffic": ncu_traffic(), "peak_kind": f"{peak_kind} bf16 (burst)",
-            "kernel": "chunk_attn_kernel",
-            "hbm_frac": round(step_bytes(w) / (ms_per_step * 1e-3) / 1e9 / peak_hbm, 4)}
-    n_sets = max(2, int(math.ceil(3 * L2_BYTES / step_bytes(w))))
+            "traffic": ncu_traffic(w.name) if not rotation_pass else None,
+            "peak_kind": f"{peak_kind} bf16 (burst)",
+            "frac_of_spec": round(per_gpu_tf / SPEC_BF16_TFLOPS, 4),
+            "spec_peak": SPEC_BF16_TFLOPS,
+            "kernel": "chunk_attn_kernel" + (" (after the rotation kernel)" if rotation_pass else ""),
+            "hbm_frac": round(step_bytes(w_rank) / (ms_per_step * 1e-3) / 1e9 / peak_hbm, 4)}
+    scaling = "strong" if ran["kind"] == "cfg" else "weak"
+    parallelism = (f"cfg{world} (rank r runs CFG branch r: batch 1 with its own cache half)"
+                   if ran["kind"] == "cfg" else f"dp{world} (independent replicas of the call)")
     line = {"metric": METRIC, "value": round(tflops, 3), "unit": "TFLOP/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_per_step, 6), "us_per_call": round(ms_per_step * 1e3, 3),
             "pct_of_bf16_peak": round(100 * per_gpu_tf / peak_tf, 2),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "pct_of_spec_bf16_peak": round(100 * per_gpu_tf / SPEC_BF16_TFLOPS, 2),
+            "higher_is_better": True, "scaling": scaling, "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic",
-            "config": dict(config, l2=f"inputs cycle through {n_sets} sets "
-                                      f"({n_sets * step_bytes(w) / 2**20:.0f} MiB > 126 MB L2)",
-                           parallelism=f"dp{world} (independent replicas of the call)"),
+            "config": dict(config, l2=f"inputs cycle through {ran['n_sets']} sets "
+                                      f"({ran['n_sets'] * ran['set_bytes'] / 2**20:.0f} MiB > "
+                                      f"126 MB L2)",
+                           parallelism=parallelism),
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps * launches_per_step(w), "clocks": clocks}
+            "gpu_launches": args.steps * launches_per_step(w, rotation_pass), "clocks": clocks}
+    if extra is not None:
+        line["workloads"] = extra
     print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    argv = sys.argv[1:]
+    args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ and args.impl == "ours":
+        spawn_ranks(args.gpus, rank_main, argv)
+        return
+    rank_main(argv)
 
 
 if __name__ == "__main__":

@@ -1,5 +1,10 @@
 """Build libdz.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
+Also builds libdz_test.so from the same sources for the device-timeout tests:
+every bounded device wait gives up after 20 ms instead of 2 s, and the library
+exports one extra call, dz_test_fill_split_counters, that presets the split
+counters so that a merge's wait can never complete.  Nothing but the tests loads it.
+
 Usage: python -m causal_video_diffusion_rope_b200.build [--verbose-ptxas]
 """
 from __future__ import annotations
@@ -13,6 +18,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdz.so")
+TEST_LIB = os.path.join(HERE, "libdz_test.so")
+TEST_DEFINES = ["-DDZ_TEST_HOOKS", "-DDZ_WAIT_NS=20000000ull"]
 SOURCES = ["dz_api.cu", "dz_kernels.cu", "dz_attn.cu", "dz_qkv.cu", "dz_bwd.cu"]
 HEADERS = ["dz_internal.cuh", "dz_ptx.cuh"]
 
@@ -24,26 +31,24 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
     deps.append(os.path.join(ROOT, "include", "dz.h"))
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
+def _compile(out: str, defines, verbose_ptxas: bool) -> None:
     cmd = [
         nvcc_path(), "-O3", "-std=c++17", "-lineinfo",
         "-gencode", "arch=compute_100a,code=sm_100a",
         "-Xcompiler", "-fPIC", "-shared",
         "-I", os.path.join(ROOT, "include"),
-        "-o", LIB + ".tmp",
-    ]
+        "-o", out + ".tmp",
+    ] + list(defines)
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     cmd += [os.path.join(CSRC, f) for f in SOURCES]
@@ -52,7 +57,15 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose_ptxas:
         sys.stderr.write(res.stderr)
-    os.replace(LIB + ".tmp", LIB)
+    os.replace(out + ".tmp", out)
+
+
+def build(force: bool = False, verbose_ptxas: bool = False, test_lib: bool = True) -> str:
+    """Compile libdz.so (and, unless test_lib is False, libdz_test.so) if stale or forced."""
+    if force or _stale(LIB):
+        _compile(LIB, [], verbose_ptxas)
+    if test_lib and (force or _stale(TEST_LIB)):
+        _compile(TEST_LIB, TEST_DEFINES, False)
     return LIB
 
 

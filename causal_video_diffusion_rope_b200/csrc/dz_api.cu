@@ -111,9 +111,22 @@ dz_status check_positions(const dz_attn* a, const dz::ChunkGeom& g, long long fi
   return DZ_OK;
 }
 
+#ifdef DZ_TEST_HOOKS
+// Test builds only (libdz_test.so): every attention call first fills its split
+// counters with this value (0 = off).  A value with zero low half and a nonzero high
+// half lets the pieces of a split unit count their arrivals as usual, while the
+// merging piece's wait for the others' publications can never complete, so the
+// bounded wait runs out and the call reports DZ_ERR_TIMEOUT.
+int g_test_counter_fill = 0;
+#endif
+
 }  // namespace
 
 extern "C" {
+
+#ifdef DZ_TEST_HOOKS
+void dz_test_fill_split_counters(int32_t value) { g_test_counter_fill = value; }
+#endif
 
 const char* dz_status_string(dz_status s) {
   switch (s) {
@@ -393,6 +406,12 @@ static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const v
       st = make_map(a, &p.tm_cv, cache->v, l->batch, cache_len, cache->capacity_tokens, H);
   }
   if (st != DZ_OK) return st;
+#ifdef DZ_TEST_HOOKS
+  if (g_test_counter_fill != 0 &&
+      dz::launch_fill_i32(a->counters, a->n_counters, g_test_counter_fill,
+                          static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return DZ_ERR_CUDA;
+#endif
   return cuda_status(dz::launch_attention(p, static_cast<cudaStream_t>(stream)),
                      "attention launch");
 }
@@ -577,8 +596,10 @@ dz_status dz_chunk_attn_backward(dz_attn_t a, const void* q, const void* k, cons
   return cuda_status(dz::launch_backward(p, static_cast<cudaStream_t>(stream)), "backward launch");
 }
 
+static dz_status noalloc_sync_status(void* stream);
+
 dz_status dz_attn_sync_status(dz_attn_t a, void* stream) {
-  if (!a) return DZ_ERR_INVALID_ARG;
+  if (!a) return noalloc_sync_status(stream);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return DZ_ERR_CUDA;
   int word = 0;
@@ -712,6 +733,10 @@ extern "C" dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* d, const 
         }
         off += static_cast<size_t>(npos[ax]) * npairs[ax];
       }
+      // earlier calls (on any stream) may still read the old tables: the device must
+      // be idle before they are overwritten, and the new ones must have landed
+      // before this call's kernels run
+      if (cudaDeviceSynchronize() != cudaSuccess) return DZ_ERR_CUDA;
       if (!tab.empty() && (cudaMemcpy(nd.rope, tab.data(), tab.size() * sizeof(float2),
                                       cudaMemcpyHostToDevice) != cudaSuccess ||
                            cudaDeviceSynchronize() != cudaSuccess))
@@ -744,11 +769,37 @@ extern "C" dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* d, const 
   a.encode = nd.encode;
   a.rot_ws = nullptr;  // no pre-rotation workspace: rotation stays inside the kernel
   a.rot_tokens = 0;
-  // the split counters and the status word must start at zero (a previous call that
-  // gave up may have left them set); cleared on the caller's stream
+  // the split counters must start at zero (a previous call that gave up may have left
+  // them set); cleared on the caller's stream.  The status word keeps a timeout until
+  // dz_attn_sync_status(NULL, stream) reads and clears it.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(a.counters, 0, a.n_counters * sizeof(int), st) != cudaSuccess ||
-      cudaMemsetAsync(a.status, 0, sizeof(int), st) != cudaSuccess)
+  if (cudaMemsetAsync(a.counters, 0, a.n_counters * sizeof(int), st) != cudaSuccess)
     return DZ_ERR_CUDA;
   return dz_chunk_attn_forward(&a, q, k, v, cache, layout, out, stream);
+}
+
+// Status of the allocation-free calls on the current device (dz_attn_sync_status
+// with a NULL handle).
+static dz_status noalloc_sync_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return DZ_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DZ_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc[dev].ready) return DZ_OK;  // no allocation-free call on this device yet
+    scratch = g_noalloc[dev].scratch;
+  }
+  int* counters = reinterpret_cast<int*>(scratch + NOALLOC_WS_BYTES);
+  int* status = reinterpret_cast<int*>(scratch + NOALLOC_WS_BYTES + NOALLOC_COUNTERS * sizeof(int));
+  int word = 0;
+  if (cudaMemcpy(&word, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DZ_ERR_CUDA;
+  if (word == 0) return DZ_OK;
+  if (cudaMemset(status, 0, sizeof(int)) != cudaSuccess ||
+      cudaMemset(counters, 0, NOALLOC_COUNTERS * sizeof(int)) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess)
+    return DZ_ERR_CUDA;
+  return DZ_ERR_TIMEOUT;
 }

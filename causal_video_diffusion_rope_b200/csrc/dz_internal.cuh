@@ -147,6 +147,10 @@ __host__ __device__ __forceinline__ int unit_tile_count(const SchedGeom& g, int 
 // ---------------------------------------------------------------------------
 cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int B, int rows,
                            int H, int cap, int dst_row0, cudaStream_t stream);
+#ifdef DZ_TEST_HOOKS
+// Test builds only: x[0:n] = value.
+cudaError_t launch_fill_i32(int* x, size_t n, int value, cudaStream_t stream);
+#endif
 
 // Rotates x into y (and x1 into y1 when x1 is not null) for B x S tokens; with
 // period > 0 token s is rotated at the position of token s % period.

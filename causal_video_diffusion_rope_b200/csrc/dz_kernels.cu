@@ -112,4 +112,19 @@ cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const Chu
   return cudaGetLastError();
 }
 
+#ifdef DZ_TEST_HOOKS
+__global__ void fill_i32_kernel(int* x, size_t n, int value) {
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x)
+    x[i] = value;
+}
+
+cudaError_t launch_fill_i32(int* x, size_t n, int value, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const unsigned blocks = static_cast<unsigned>(n / 256 + 1 < 1024 ? n / 256 + 1 : 1024);
+  fill_i32_kernel<<<blocks, 256, 0, stream>>>(x, n, value);
+  return cudaGetLastError();
+}
+#endif
+
 }  // namespace dz

@@ -78,15 +78,8 @@ class dz_kvcache(ctypes.Structure):
 _lib: Optional[ctypes.CDLL] = None
 
 
-def load() -> ctypes.CDLL:
-    """Load libdz.so from the package directory (raises if it is not built)."""
-    global _lib
-    if _lib is not None:
-        return _lib
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libdz.so is not built ({LIB_PATH}); run "
-                          "python -m causal_video_diffusion_rope_b200.build")
-    lib = ctypes.CDLL(LIB_PATH)
+def bind(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the argument and result types of every entry point on a loaded libdz."""
     vp, i32 = ctypes.c_void_p, ctypes.c_int32
     lib.dz_attn_create.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(dz_attn_desc)]
     lib.dz_attn_destroy.argtypes = [vp]
@@ -110,8 +103,19 @@ def load() -> ctypes.CDLL:
     for name in EXPORTS:
         if name != "dz_status_string":
             getattr(lib, name).restype = ctypes.c_int
-    _lib = lib
     return lib
+
+
+def load() -> ctypes.CDLL:
+    """Load libdz.so from the package directory (raises if it is not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libdz.so is not built ({LIB_PATH}); run "
+                          "python -m causal_video_diffusion_rope_b200.build")
+    _lib = bind(ctypes.CDLL(LIB_PATH))
+    return _lib
 
 
 def status_string(status: int) -> str:

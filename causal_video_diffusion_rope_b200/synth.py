@@ -225,3 +225,13 @@ def fresh_chunk(rng: np.random.Generator, w: Workload) -> Dict[str, np.ndarray]:
         "k": normal_bf16(rng, (B, lay.self_kv_len, H, D)),
         "v": normal_bf16(rng, (B, lay.self_kv_len, H, D)),
     }
+
+
+def branch_inputs(w: Workload, inp: Dict[str, np.ndarray], branch: int):
+    """One batch item (a CFG branch) of a workload and its inputs: the workload with
+    batch 1 and every batched tensor sliced to item ``branch`` (its own cache half)."""
+    lay = dataclasses.replace(w.layout, batch=1)
+    wb = dataclasses.replace(w, layout=lay)
+    out = {k: (v[branch:branch + 1] if k != "boosted_heads" else v) for k, v in inp.items()}
+    return wb, out
+

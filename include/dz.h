@@ -283,19 +283,25 @@ dz_status dz_qkv_rope(dz_attn_t handle, const void* x, const void* w, int32_t B,
  * the split uses at most 63 CTAs, so large calls run slower than through a
  * handle.  The first call on a device looks up the arrays' device addresses,
  * and the first call with a given rotary configuration (base, pairs, max_pos)
- * fills the tables with a synchronous copy: make those calls before any stream
- * capture.  Every call clears the split counters on `stream` and then uses the
- * same arrays, which keep the last call's contents: calls that overlap on the
- * GPU (other streams, other threads) race and give wrong results.  Device-side
- * timeouts are not reported on this path.  Arguments as dz_chunk_attn_forward,
- * with desc in place of the handle. */
+ * waits until the device is idle (earlier calls may still read the old tables)
+ * and then fills the tables with a synchronous copy: make those calls before
+ * any stream capture.  Every call clears the split counters on `stream` and
+ * then uses the same arrays, which keep the last call's contents: calls that
+ * overlap on the GPU (other streams, other threads) race and give wrong
+ * results.  A device-side timeout (a bounded wait that ran out, leaving `out`
+ * incomplete) is kept in the static status word until dz_attn_sync_status(NULL,
+ * stream) reads and clears it.  Arguments as dz_chunk_attn_forward, with desc
+ * in place of the handle. */
 dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* desc, const void* q, const void* k,
                                         const void* v, const dz_kvcache* cache,
                                         const dz_chunk_layout* layout, void* out, void* stream);
 
 /* Synchronise `stream`, read and clear the handle's device status word.
  * Returns DZ_ERR_TIMEOUT if a kernel's bounded wait ran out since the last
- * read, DZ_ERR_CUDA on a CUDA error, else DZ_OK. */
+ * read (that call's output is incomplete), DZ_ERR_CUDA on a CUDA error, else
+ * DZ_OK.  With a NULL handle it reads and clears the status word of the
+ * allocation-free calls (dz_chunk_attn_forward_noalloc) on the current device
+ * instead (DZ_OK if none was made there). */
 dz_status dz_attn_sync_status(dz_attn_t handle, void* stream);
 
 /* Static English name of a status code. */

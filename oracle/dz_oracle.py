@@ -31,7 +31,7 @@ Sources (page title, section):
   * Cross-attention to the concatenated visual + language conditioning --
     "DreamZero (WAM) 模型架构", §2.1 (fusion diagram) and §2.3 block diagram.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * mask granularity is the chunk; inside a chunk attention is bidirectional;
     action tokens follow their chunk's rule;
   * teacher forcing: clean chunk i sees clean chunks <= i; noisy chunk i sees

@@ -72,7 +72,9 @@ def test_calls_reject_null_handle(lib):
     assert lib.dz_kvcache_append(None, ctypes.byref(cache), 16, 16, None) == dz.DZ_ERR_INVALID_ARG
     assert lib.dz_kvcache_replace(None, ctypes.byref(cache), 0, 16, 16, None) == \
         dz.DZ_ERR_INVALID_ARG
-    assert lib.dz_attn_sync_status(None, None) == dz.DZ_ERR_INVALID_ARG
+    # a NULL handle asks for the allocation-free calls' status word: without a device the
+    # stream synchronisation fails, on a device with no such call yet it is clear
+    assert lib.dz_attn_sync_status(None, None) in (dz.DZ_OK, dz.DZ_ERR_CUDA)
     assert lib.dz_attn_destroy(None) == dz.DZ_ERR_INVALID_ARG
     pre = dz.make_layout(dz.DZ_MODE_PREFILL, 1, 1, 4, 4, 4, 2)
     assert lib.dz_qkv_rope(None, 16, 16, 1, 20, 128, ctypes.byref(pre), 0, 16, 16, 16, None,
