@@ -522,12 +522,13 @@ class AttnSetup:
         self.sets.clear()
 
 
-def extra_workload_block(wl: int, dev, stream, steps: int, peak_tf: float, peak_hbm: float):
+def extra_workload_block(wl: int, dev, stream, steps: int, peak_tf: float, peak_hbm: float,
+                         rotation_pass: bool):
     """Timing of one more full-size workload (N=1), the headline's discipline: graphs of
     calls cycling input sets above L2, CUDA events on the launching stream."""
     import torch
     w = synth.WORKLOADS[wl]
-    st = AttnSetup(w, dev, 2000 + 100 * wl, rotation_pass=False, max_sets=3)
+    st = AttnSetup(w, dev, 2000 + 100 * wl, rotation_pass=rotation_pass, max_sets=3)
     n = max(20, min(steps, 240))
     res = {"workload": w.name, "mode": synth.MODE_NAMES[w.layout.mode],
            "batch": w.layout.batch, "q_tokens": w.layout.q_len,
@@ -621,7 +622,7 @@ def run_attention(args, rank: int, world: int, local_rank: int):
     extra = None
     if world == 1 and args.extra:
         peak_tf, peak_hbm, _ = measured_peaks()
-        extra = [extra_workload_block(x, dev, stream, args.steps, peak_tf, peak_hbm)
+        extra = [extra_workload_block(x, dev, stream, args.steps, peak_tf, peak_hbm, rotation_pass)
                  for x in EXTRA_WORKLOADS if x != args.workload]
     return ms_per_step, tflops_total, clocks, e2e, ran, extra
 
@@ -891,7 +892,7 @@ def parse_args(argv):
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
                     choices=range(len(synth.WORKLOADS)),
                     help="workload index (default: the single-layer inference step)")
-    ap.add_argument("--rotation", default="kernel", choices=["kernel", "pass"],
+    ap.add_argument("--rotation", default="pass", choices=["kernel", "pass"],
                     help="kernel: q and the chunk's k rotated as the attention kernel loads "
                          "them; pass: rotated once per call by a separate kernel first")
     ap.add_argument("--no-extra", dest="extra", action="store_false",

@@ -122,10 +122,101 @@ int g_test_counter_fill = 0;
 
 }  // namespace
 
+namespace dz {
+
+// Work split of an attention call over at most num_sms CTAs.
+//  * One CTA per unit (no split) when the units fit the SMs and splitting would not
+//    shorten the longest CTA by more than its merge costs.
+//  * Otherwise `waves` rounds of whole units first, unit c + k * grid going to CTA c
+//    (head-major order: the CTAs that run together work on the same few heads, whose
+//    keys then come from L2), used when there is at least one full wave and the rest
+//    is at least half a wave and no CTA's whole units exceed its balanced share; then
+//    the remaining units' key tiles, cut into one contiguous range per CTA so that
+//    every CTA ends up with the same estimated work (tiles plus a start-up cost per
+//    whole unit).  A unit whose tiles fall in several ranges is merged from pieces.
+void plan_schedule(AttnLaunch& a, const int* T, int n_qg, long long bh_count, int num_sms) {
+  const long long units = bh_count * n_qg;
+  long long per_bh = 0;
+  int t_max = 0;
+  for (int qg = 0; qg < n_qg; ++qg) {
+    per_bh += T[qg];
+    if (T[qg] > t_max) t_max = T[qg];
+  }
+  const long long W = per_bh * bh_count;
+  const int sms = num_sms < MAX_GRID ? num_sms : MAX_GRID;
+  const long long split_tiles = (W + sms - 1) / sms;
+  if (units <= sms && t_max <= split_tiles + SPLIT_OVERHEAD_TILES) {
+    a.grid = static_cast<int>(units);
+    a.waves = 1;
+    for (int c = 0; c <= a.grid; ++c) a.tb[c] = static_cast<unsigned>(W);  // no tail
+    return;
+  }
+  const int G = static_cast<int>(W < sms ? W : sms);
+  a.grid = G;
+  int waves = 0;
+  std::vector<double> R(G, 0.0);
+  double target = static_cast<double>(W) / G;
+  for (long long k = units / G; k >= 1; --k) {
+    if (units - k * G < G / 2) continue;
+    std::vector<double> r(G, 0.0);
+    long long wave_tiles = 0;
+    for (long long u = 0; u < k * G; ++u) {
+      const int t = T[u % n_qg];
+      wave_tiles += t;
+      r[u % G] += t + UNIT_SWITCH_TILES;
+    }
+    double tot = static_cast<double>(W - wave_tiles), rmax = 0.0;
+    for (int c = 0; c < G; ++c) {
+      tot += r[c];
+      if (r[c] > rmax) rmax = r[c];
+    }
+    if (rmax <= tot / G) {
+      waves = static_cast<int>(k);
+      R = r;
+      target = tot / G;
+      break;
+    }
+  }
+  a.waves = waves;
+  long long P0 = 0;  // flattened position of the first unit of the tail
+  for (long long u = 0; u < static_cast<long long>(waves) * G; ++u) P0 += T[u % n_qg];
+  const long long tail = W - P0;
+  a.tb[0] = static_cast<unsigned>(P0);
+  if (waves == 0) {
+    for (int c = 1; c <= G; ++c) a.tb[c] = static_cast<unsigned>(c * W / G);
+  } else {
+    double sum = 0.0;
+    for (int c = 0; c < G; ++c) sum += target - R[c] > 0.0 ? target - R[c] : 0.0;
+    double cum = 0.0;
+    for (int c = 0; c < G; ++c) {
+      cum += (target - R[c] > 0.0 ? target - R[c] : 0.0) * (static_cast<double>(tail) / sum);
+      long long b = P0 + static_cast<long long>(cum);
+      if (b > W) b = W;
+      a.tb[c + 1] = static_cast<unsigned>(b);
+    }
+    a.tb[G] = static_cast<unsigned>(W);
+  }
+}
+
+}  // namespace dz
+
 extern "C" {
 
 #ifdef DZ_TEST_HOOKS
 void dz_test_fill_split_counters(int32_t value) { g_test_counter_fill = value; }
+
+// The work split of an attention call for `bh_count` (batch, head) pairs whose query
+// groups have tiles[0 .. n_qg) key tiles each, over at most num_sms CTAs: writes the
+// grid, the number of whole-unit waves and the tail ranges (grid + 1 entries of tb).
+int32_t dz_test_plan_schedule(const int32_t* tiles, int32_t n_qg, int64_t bh_count,
+                              int32_t num_sms, int32_t* grid, int32_t* waves, uint32_t* tb) {
+  static dz::AttnLaunch a;
+  dz::plan_schedule(a, tiles, n_qg, bh_count, num_sms);
+  *grid = a.grid;
+  *waves = a.waves;
+  for (int c = 0; c <= a.grid; ++c) tb[c] = a.tb[c];
+  return 0;
+}
 #endif
 
 const char* dz_status_string(dz_status s) {
@@ -335,29 +426,17 @@ static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const v
   p.sched.nks = cdiv(static_cast<int>(Sk), dz::TILE_N);
   p.n_qg = cdiv(static_cast<int>(Sq), dz::Q_GROUP);
   if (p.n_qg > dz::MAX_Q_GROUPS) return DZ_ERR_CAPACITY;
+  std::vector<int> tiles(p.n_qg);
   long long per_bh = 0;
-  for (int qg = 0; qg < p.n_qg; ++qg) per_bh += dz::unit_tile_count(p.sched, qg);
-  p.W = per_bh * l->batch * H;
-  if (p.W <= 0) return DZ_ERR_SHAPE;
-  // Work split: split units across CTAs (stream-K, with a merge of partial results)
-  // only when that shortens the longest CTA by more than the merge costs; a unit that
-  // one CTA runs whole writes its output directly.
-  {
-    const long long units = static_cast<long long>(l->batch) * H * p.n_qg;
-    int t_max = 0;
-    for (int qg = 0; qg < p.n_qg; ++qg) {
-      const int t = dz::unit_tile_count(p.sched, qg);
-      if (t > t_max) t_max = t;
-    }
-    const long long split_tiles = (p.W + a->num_sms - 1) / a->num_sms;
-    if (units <= a->num_sms && t_max <= split_tiles + dz::SPLIT_OVERHEAD_TILES) {
-      p.grid = static_cast<int>(units);
-    } else {
-      p.grid = static_cast<int>(p.W < a->num_sms ? p.W : a->num_sms);
-    }
+  for (int qg = 0; qg < p.n_qg; ++qg) {
+    tiles[qg] = dz::unit_tile_count(p.sched, qg);
+    per_bh += tiles[qg];
   }
+  const long long W = per_bh * l->batch * H;
+  if (W <= 0) return DZ_ERR_SHAPE;
   // the kernel schedules key tiles with 32-bit arithmetic
-  if (p.W * (p.grid + 1LL) >= (1LL << 31)) return DZ_ERR_UNSUPPORTED;
+  if (W >= (1LL << 31)) return DZ_ERR_UNSUPPORTED;
+  dz::plan_schedule(p, tiles.data(), p.n_qg, static_cast<long long>(l->batch) * H, a->num_sms);
   p.B = l->batch;
   p.H = H;
   p.geom = g;

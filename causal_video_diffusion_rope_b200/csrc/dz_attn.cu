@@ -26,10 +26,12 @@
 // (log2 domain) and rescales O only when m grows by more than 8 (factor 256);
 // the final O / l uses the same m, so the result is exact up to rounding.
 //
-// Work split (stream-K): unit = (batch, head, group of 256 query rows); its
-// key tiles are the tiles any of its rows can see (fully masked tiles are never
-// loaded).  All units' tiles are laid end to end and cut into one contiguous
-// range per CTA (one CTA per unit when that is no slower).  A unit that one
+// Work split: unit = (batch, head, group of 256 query rows); its key tiles are
+// the tiles any of its rows can see (fully masked tiles are never loaded).  With
+// many units, whole units are first dealt round-robin in head-major order (the
+// CTAs that run together share the same heads' keys through L2); the remaining
+// units' tiles are laid end to end and cut into one contiguous range per CTA
+// (stream-K; one CTA per unit when that is no slower).  A unit that one
 // CTA covers entirely writes bf16 output directly; otherwise each piece counts
 // its arrival on the unit's counter, every piece but the last to arrive
 // publishes fp32 partial (O, m, l) to the workspace, and the last one merges
@@ -107,8 +109,9 @@ struct __align__(64) AttnParams {
   int B, H, n_qg;
   int rope_q, rope_k;
   int stage_ok, stage_t0, stage_nt;
-  unsigned W;  // total key tiles; W * G < 2^31 (checked on the host)
-  int G;
+  int G;      // CTAs
+  int waves;  // rounds of whole units dealt round-robin before the split tail
+  unsigned tb[MAX_GRID + 1];  // tail: CTA c holds flattened key tiles [tb[c], tb[c + 1])
   float scale_log2;
 };
 
@@ -121,10 +124,40 @@ struct Seg {
   unsigned u0, u1;  // flattened tile range of the unit
 };
 
-__device__ __forceinline__ bool seg_next(const AttnParams& p, const int* prefix, unsigned& pos,
+// Where a CTA is in its work list: k whole units dealt so far, then the position in
+// its tail range.
+struct Cursor {
+  int k;
+  unsigned pos;
+};
+
+// The CTA's next segment.  First `waves` whole units, unit blockIdx.x + k * G of the
+// head-major unit order (the CTAs that run together work on the same few heads and
+// read their keys from L2), then its contiguous range of the remaining units' key
+// tiles, whose units may be split across CTAs.
+__device__ __forceinline__ bool seg_next(const AttnParams& p, const int* prefix, Cursor& cur,
                                          unsigned end, Seg& s) {
-  if (pos >= end) return false;
   const int Tbh = prefix[p.n_qg];
+  if (cur.k < p.waves) {
+    const int u = static_cast<int>(blockIdx.x) + cur.k * p.G;
+    ++cur.k;
+    const int bh = u / p.n_qg, qg = u - (u / p.n_qg) * p.n_qg;
+    const int Tq = prefix[qg + 1] - prefix[qg];
+    s.bh = bh;
+    s.qg = qg;
+    s.t0 = 0;
+    s.n = Tq;
+    s.full = true;
+    s.u0 = static_cast<unsigned>(bh) * Tbh + prefix[qg];
+    s.u1 = s.u0 + Tq;
+    int e1, s2, e2;
+    unit_tiles(p.sched, qg, e1, s2, e2);
+    s.e1 = e1;
+    s.s2 = s2;
+    return true;
+  }
+  unsigned& pos = cur.pos;
+  if (pos >= end) return false;
   const unsigned bh = pos / static_cast<unsigned>(Tbh);
   const int rem = static_cast<int>(pos - bh * Tbh);
   int lo = 0, hi = p.n_qg - 1;  // largest qg with prefix[qg] <= rem
@@ -330,12 +363,14 @@ __device__ __forceinline__ void rotate_tile_row_split(uint32_t tile, int r, uint
   }
 }
 
-__device__ __forceinline__ unsigned cta_start(unsigned c, unsigned W, int G) {
-  return c * W / static_cast<unsigned>(G);
-}
-// The CTA whose range holds flattened tile x.
-__device__ __forceinline__ int cta_of(unsigned x, unsigned W, int G) {
-  return static_cast<int>(((x + 1) * static_cast<unsigned>(G) - 1) / W);
+// The CTA whose tail range holds flattened tile x: the largest c with tb[c] <= x.
+__device__ __forceinline__ int cta_of(const AttnParams& p, unsigned x) {
+  int lo = 0, hi = p.G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (p.tb[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
 
@@ -430,15 +465,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const unsigned cstart = cta_start(blockIdx.x, p.W, p.G);
-  const unsigned cend = cta_start(blockIdx.x + 1, p.W, p.G);
+  const Cursor cstart = {0, p.tb[blockIdx.x]};
+  const unsigned cend = p.tb[blockIdx.x + 1];
 
   if (warp < WARP_SOFT) {
   regs_dec<REGS_CTRL>();
   if (warp == WARP_TMA) {
     // ======================= TMA producer =======================
     if (lane == 0) {
-      unsigned pos = cstart;
+      Cursor pos = cstart;
       Seg sg;
       int seg_i = 0;
       uint32_t k_iss = 0, v_iss = 0;  // K and V tiles issued so far
@@ -515,7 +550,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  (acc || kk > 0) ? 1u : 0u);
         }
       };
-      unsigned pos = cstart;
+      Cursor pos = cstart;
       Seg sg;
       int seg_i = 0;
       uint32_t it = 0, tn = 0;
@@ -613,7 +648,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         rotate_tile_row(tile, r, rope, t, h, w);
       }
     };
-    unsigned pos = cstart;
+    Cursor pos = cstart;
     Seg sg;
     int seg_i = 0;
     uint32_t it = 0;
@@ -664,7 +699,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tO = tmem + lane_addr + 256 + q * HEAD_DIM;
     uint8_t* xp = smem + SM_X + (warp - WARP_SOFT) * XPOSE_WARP;  // this warp's transpose buffer
     const float sl2 = p.scale_log2;
-    unsigned pos = cstart;
+    Cursor pos = cstart;
     Seg sg;
     int seg_i = 0;
     uint32_t tn = 0;
@@ -783,12 +818,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // row as float2.
         constexpr int ROWS = Q_TILES * TILE_M;
         const int row_l = q * TILE_M + r;
-        const int c_first = cta_of(sg.u0, p.W, p.G);
-        const int c_last = cta_of(sg.u1 - 1, p.W, p.G);
+        const int c_first = cta_of(p, sg.u0);
+        const int c_last = cta_of(p, sg.u1 - 1);
         const int np = c_last - c_first + 1;
         // slot of the piece held by CTA c: its first segment (slot 2c) unless the
         // unit began before c's range, which only the first piece's CTA can see
-        const int slot0 = 2 * c_first + (cta_start(c_first, p.W, p.G) == sg.u0 ? 0 : 1);
+        const int slot0 = 2 * c_first + (p.tb[c_first] == sg.u0 ? 0 : 1);
         const int me = static_cast<int>(blockIdx.x) - c_first;  // piece index
         auto slot_of = [&](int k) { return k == 0 ? slot0 : 2 * (c_first + k); };
         int* counter = p.counters + (static_cast<size_t>(sg.bh) * p.n_qg + sg.qg) * Q_TILES + q;
@@ -969,8 +1004,9 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   p.stage_ok = a.stage_ok;
   p.stage_t0 = a.stage_t0;
   p.stage_nt = a.stage_nt;
-  p.W = static_cast<unsigned>(a.W);
   p.G = a.grid;
+  p.waves = a.waves;
+  for (int c = 0; c <= a.grid; ++c) p.tb[c] = a.tb[c];
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));
   chunk_attn_kernel<<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
   return cudaGetLastError();

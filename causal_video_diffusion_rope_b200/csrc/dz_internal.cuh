@@ -15,6 +15,7 @@ constexpr int TILE_N = 128;        // keys per K/V tile
 constexpr int Q_TILES = 2;         // Q tiles per CTA (ping-pong between two softmax groups)
 constexpr int Q_GROUP = TILE_M * Q_TILES;  // query rows per work unit
 constexpr int MAX_Q_GROUPS = 512;  // per (batch, head); bounds the per-CTA prefix table
+constexpr int MAX_GRID = 512;      // CTAs of one attention launch (the schedule is a kernel parameter)
 
 // Rotary tables: (cos, sin) as float2 for every (axis position, pair of that axis).
 struct RopeTables {
@@ -174,13 +175,25 @@ struct AttnLaunch {
   // rotary-table rows the call needs (t in [stage_t0, stage_t0 + stage_nt), all h < gh,
   // all w < gw), copied to shared memory at kernel start when stage_ok
   int stage_ok, stage_t0, stage_nt;
-  long long W;  // total key tiles over all units
+  // Schedule over `grid` CTAs: `waves` rounds of whole units dealt round-robin (CTA c
+  // takes unit c + k * grid of the head-major order), then CTA c takes the flattened
+  // key tiles [tb[c], tb[c + 1]) of the remaining units, splitting units between CTAs.
   int grid;
+  int waves;
+  unsigned tb[MAX_GRID + 1];
 };
+
+// Schedule of an attention call (see AttnLaunch): fills grid, waves and tb from the
+// tile counts of the query groups of one (batch, head), `units_bh` groups each.
+void plan_schedule(AttnLaunch& a, const int* tiles_per_qg, int n_qg, long long bh_count,
+                   int num_sms);
 
 // Cost of splitting a unit across CTAs (partial write, merge, extra Q loads), in
 // key tiles: a call runs one unit per CTA unless splitting saves more than this.
 constexpr int SPLIT_OVERHEAD_TILES = 10;
+// Estimated cost of starting a unit (Q load, pipeline fill, epilogue), in key tiles,
+// used to balance the whole units of the round-robin waves against the tail.
+constexpr int UNIT_SWITCH_TILES = 2;
 
 // Capacity (float2 entries) of the attention kernel's shared-memory rotary table.
 constexpr int ROPE_STAGE_MAX = 1280;
