@@ -678,6 +678,16 @@ def run_qkv(args, rank: int, world: int, local_rank: int, config: dict):
     ms_ref, _ = time_graph(stream, call_ref, min(args.steps, 2400), 3, world, dev)
     ref_us = 1e3 * ms_ref / min(args.steps, 2400)
 
+    # the rotation the unfused path adds after that GEMM: q and k through dz_rope3d
+    qr, kr = torch.empty_like(q), torch.empty_like(k)
+
+    def call_rot(i):
+        dz.dz_rope3d(h, q, qr, B, S, dl, first, stream)
+        dz.dz_rope3d(h, k, kr, B, S, dl, first, stream)
+
+    ms_rot, _ = time_graph(stream, call_rot, min(args.steps, 2400), 3, world, dev)
+    rot_us = 1e3 * ms_rot / min(args.steps, 2400)
+
     def e2e_call(di, do):
         dz.dz_qkv_rope(h, di["x"], W, B, S, D_MODEL, dl, first, do["q"], do["k"], do["v"],
                        None, stream)
@@ -705,7 +715,9 @@ def run_qkv(args, rank: int, world: int, local_rank: int, config: dict):
                          "unit": "TFLOP/s", "frac": round(per_gpu / peak_tf, 4), "traffic": None,
                          "peak_kind": f"{peak_kind} bf16 (burst)", "kernel": "qkv_rope_kernel"},
             "context": {"cublas_same_gemm_us": round(ref_us, 3),
-                        "cublas_same_gemm_tflops": round(flops / (ref_us * 1e-6) / 1e12, 2)},
+                        "cublas_same_gemm_tflops": round(flops / (ref_us * 1e-6) / 1e12, 2),
+                        "rotation_pass_us": round(rot_us, 3),
+                        "unfused_us": round(ref_us + rot_us, 3)},
             "cpu_baseline": None, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks}
     print(json.dumps(line), flush=True)
 

@@ -21,7 +21,7 @@ LIB = os.path.join(HERE, "libdz.so")
 TEST_LIB = os.path.join(HERE, "libdz_test.so")
 TEST_DEFINES = ["-DDZ_TEST_HOOKS", "-DDZ_WAIT_NS=20000000ull"]
 SOURCES = ["dz_api.cu", "dz_kernels.cu", "dz_attn.cu", "dz_qkv.cu", "dz_bwd.cu"]
-HEADERS = ["dz_internal.cuh", "dz_ptx.cuh"]
+HEADERS = ["dz_internal.cuh", "dz_ops.cuh", "dz_ptx.cuh"]
 
 
 def nvcc_path() -> str:

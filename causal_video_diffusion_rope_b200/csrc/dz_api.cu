@@ -11,7 +11,7 @@
 #include <vector>
 
 #include "../../include/dz.h"
-#include "dz_internal.cuh"
+#include "dz_ops.cuh"
 
 struct dz_attn {
   int device;
@@ -143,12 +143,17 @@ void plan_schedule(AttnLaunch& a, const int* T, int n_qg, long long bh_count, in
     if (T[qg] > t_max) t_max = T[qg];
   }
   const long long W = per_bh * bh_count;
+  a.W = W;
+  // Units of equal size (decode, cross-attention, one query group per head) are
+  // already whole in the plain contiguous split; only ragged ones use waves.
+  const bool uniform = t_max * n_qg == per_bh;
   const int sms = num_sms < MAX_GRID ? num_sms : MAX_GRID;
   const long long split_tiles = (W + sms - 1) / sms;
   if (units <= sms && t_max <= split_tiles + SPLIT_OVERHEAD_TILES) {
     a.grid = static_cast<int>(units);
-    a.waves = 1;
-    for (int c = 0; c <= a.grid; ++c) a.tb[c] = static_cast<unsigned>(W);  // no tail
+    a.waves = uniform ? 0 : 1;
+    for (int c = 0; c <= a.grid; ++c)  // one unit per CTA, no tail
+      a.tb[c] = static_cast<unsigned>(uniform ? c * W / a.grid : W);
     return;
   }
   const int G = static_cast<int>(W < sms ? W : sms);
@@ -156,7 +161,7 @@ void plan_schedule(AttnLaunch& a, const int* T, int n_qg, long long bh_count, in
   int waves = 0;
   std::vector<double> R(G, 0.0);
   double target = static_cast<double>(W) / G;
-  for (long long k = units / G; k >= 1; --k) {
+  for (long long k = uniform ? 0 : units / G; k >= 1; --k) {
     if (units - k * G < G / 2) continue;
     std::vector<double> r(G, 0.0);
     long long wave_tiles = 0;
@@ -578,7 +583,8 @@ dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int3
     p.cache_cap = cache->capacity_tokens;
     p.cache_row0 = cache->len_tokens;
   }
-  // x as [M][d_model] and w as [N][d_model], both with 64 x 256 boxes
+  // x as [M][d_model] with 64 x 256 boxes, w as [N][d_model] with 64 x bn boxes
+  p.bn = dz::qkv_tile_n(M, N, a->num_sms);
   auto map2d = [&](CUtensorMap* m, const void* base, long long rows, int box_rows) {
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(d_model), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(d_model) * 2};
@@ -591,7 +597,7 @@ dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int3
     return r == CUDA_SUCCESS ? DZ_OK : DZ_ERR_CUDA;
   };
   st = map2d(&p.tm_x, x, M, 256);
-  if (st == DZ_OK) st = map2d(&p.tm_w, w, N, 256);
+  if (st == DZ_OK) st = map2d(&p.tm_w, w, N, p.bn);
   if (st != DZ_OK) return st;
   p.q = q_out;
   p.k = k_out;

@@ -26,17 +26,20 @@
 // (log2 domain) and rescales O only when m grows by more than 8 (factor 256);
 // the final O / l uses the same m, so the result is exact up to rounding.
 //
-// Work split: unit = (batch, head, group of 256 query rows); its key tiles are
-// the tiles any of its rows can see (fully masked tiles are never loaded).  With
-// many units, whole units are first dealt round-robin in head-major order (the
-// CTAs that run together share the same heads' keys through L2); the remaining
-// units' tiles are laid end to end and cut into one contiguous range per CTA
-// (stream-K; one CTA per unit when that is no slower).  A unit that one
+// Work split (stream-K): unit = (batch, head, group of 256 query rows); its
+// key tiles are the tiles any of its rows can see (fully masked tiles are never
+// loaded).  All units' tiles are laid end to end and cut into one contiguous
+// range per CTA (one CTA per unit when that is no slower).  Prefill and teacher
+// forcing calls with many units first deal whole units round-robin in head-major
+// order (a second instantiation of the kernel), so that the CTAs running together
+// share a few heads' keys through L2, and split only the remaining units.  A unit that one
 // CTA covers entirely writes bf16 output directly; otherwise each piece counts
 // its arrival on the unit's counter, every piece but the last to arrive
 // publishes fp32 partial (O, m, l) to the workspace, and the last one merges
 // them into its own O in TMEM.  With the call's q and own k rotated once into a
 // workspace beforehand (or given rotated), the rotary gate only passes tiles on.
+#include <type_traits>
+
 #include "dz_internal.cuh"
 #include "dz_ptx.cuh"
 
@@ -90,7 +93,8 @@ enum {
 };
 constexpr int SM_MISC = SM_BAR + 256;         // tmem base, abort flag, combine flags
 constexpr int SM_PREFIX = SM_MISC + 256;      // (MAX_Q_GROUPS + 1) ints
-constexpr int SM_ROPE = SM_PREFIX + ((MAX_Q_GROUPS + 1) * 4 + 15) / 16 * 16;  // staged rotary rows
+constexpr int SM_TB = SM_PREFIX + ((MAX_Q_GROUPS + 1) * 4 + 15) / 16 * 16;  // tail ranges (G + 1)
+constexpr int SM_ROPE = SM_TB + ((MAX_GRID + 1) * 4 + 15) / 16 * 16;  // staged rotary rows
 constexpr int SM_TOTAL = SM_ROPE + ROPE_STAGE_MAX * 8;
 constexpr int SMEM_BYTES = SM_TOTAL + 1024;   // alignment slack
 static_assert(B_COUNT * 8 <= 256, "barrier area");
@@ -109,10 +113,19 @@ struct __align__(64) AttnParams {
   int B, H, n_qg;
   int rope_q, rope_k;
   int stage_ok, stage_t0, stage_nt;
-  int G;      // CTAs
-  int waves;  // rounds of whole units dealt round-robin before the split tail
-  unsigned tb[MAX_GRID + 1];  // tail: CTA c holds flattened key tiles [tb[c], tb[c + 1])
+  unsigned W;  // total key tiles; W * G < 2^31 (checked on the host)
+  int G;
   float scale_log2;
+};
+
+// Parameters of the schedule with whole-unit waves (prefill / teacher forcing):
+// `waves` rounds of whole units dealt round-robin (CTA c takes unit c + k * G of the
+// head-major order, so the CTAs that run together read the same few heads' keys
+// and those come from L2), then CTA c takes flattened key tiles [tb[c], tb[c + 1])
+// of the remaining units.
+struct __align__(64) AttnParamsWaves : AttnParams {
+  int waves;
+  unsigned tb[MAX_GRID + 1];
 };
 
 // One contiguous piece of a unit's key-tile list handled by this CTA.
@@ -124,37 +137,38 @@ struct Seg {
   unsigned u0, u1;  // flattened tile range of the unit
 };
 
-// Where a CTA is in its work list: k whole units dealt so far, then the position in
-// its tail range.
+// Where a CTA is in its work list: whole units dealt so far (waves schedule), then
+// its position in its range of flattened key tiles.
 struct Cursor {
   int k;
   unsigned pos;
 };
 
-// The CTA's next segment.  First `waves` whole units, unit blockIdx.x + k * G of the
-// head-major unit order (the CTAs that run together work on the same few heads and
-// read their keys from L2), then its contiguous range of the remaining units' key
-// tiles, whose units may be split across CTAs.
-__device__ __forceinline__ bool seg_next(const AttnParams& p, const int* prefix, Cursor& cur,
+// The CTA's next segment: with the waves schedule first its whole units, then (both
+// schedules) the pieces of its contiguous range of flattened key tiles.
+template <class P>
+__device__ __forceinline__ bool seg_next(const P& p, const int* prefix, Cursor& cur,
                                          unsigned end, Seg& s) {
   const int Tbh = prefix[p.n_qg];
-  if (cur.k < p.waves) {
-    const int u = static_cast<int>(blockIdx.x) + cur.k * p.G;
-    ++cur.k;
-    const int bh = u / p.n_qg, qg = u - (u / p.n_qg) * p.n_qg;
-    const int Tq = prefix[qg + 1] - prefix[qg];
-    s.bh = bh;
-    s.qg = qg;
-    s.t0 = 0;
-    s.n = Tq;
-    s.full = true;
-    s.u0 = static_cast<unsigned>(bh) * Tbh + prefix[qg];
-    s.u1 = s.u0 + Tq;
-    int e1, s2, e2;
-    unit_tiles(p.sched, qg, e1, s2, e2);
-    s.e1 = e1;
-    s.s2 = s2;
-    return true;
+  if constexpr (std::is_same<P, AttnParamsWaves>::value) {
+    if (cur.k < p.waves) {
+      const int u = static_cast<int>(blockIdx.x) + cur.k * p.G;
+      ++cur.k;
+      const int bh = u / p.n_qg, qg = u - (u / p.n_qg) * p.n_qg;
+      const int Tq = prefix[qg + 1] - prefix[qg];
+      s.bh = bh;
+      s.qg = qg;
+      s.t0 = 0;
+      s.n = Tq;
+      s.full = true;
+      s.u0 = static_cast<unsigned>(bh) * Tbh + prefix[qg];
+      s.u1 = s.u0 + Tq;
+      int e1, s2, e2;
+      unit_tiles(p.sched, qg, e1, s2, e2);
+      s.e1 = e1;
+      s.s2 = s2;
+      return true;
+    }
   }
   unsigned& pos = cur.pos;
   if (pos >= end) return false;
@@ -363,12 +377,19 @@ __device__ __forceinline__ void rotate_tile_row_split(uint32_t tile, int r, uint
   }
 }
 
-// The CTA whose tail range holds flattened tile x: the largest c with tb[c] <= x.
-__device__ __forceinline__ int cta_of(const AttnParams& p, unsigned x) {
-  int lo = 0, hi = p.G - 1;
+__device__ __forceinline__ unsigned cta_start(unsigned c, unsigned W, int G) {
+  return c * W / static_cast<unsigned>(G);
+}
+// The CTA whose range holds flattened tile x.
+__device__ __forceinline__ int cta_of(unsigned x, unsigned W, int G) {
+  return static_cast<int>(((x + 1) * static_cast<unsigned>(G) - 1) / W);
+}
+// The same with explicit ranges (staged in shared memory): the largest c with tb[c] <= x.
+__device__ __forceinline__ int cta_of(const unsigned* tb, int G, unsigned x) {
+  int lo = 0, hi = G - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
-    if (p.tb[mid] <= x) lo = mid; else hi = mid - 1;
+    if (tb[mid] <= x) lo = mid; else hi = mid - 1;
   }
   return lo;
 }
@@ -376,8 +397,10 @@ __device__ __forceinline__ int cta_of(const AttnParams& p, unsigned x) {
 
 }  // namespace
 
+template <class P>
 __global__ void __launch_bounds__(NTHREADS, 1)
-    chunk_attn_kernel(const __grid_constant__ AttnParams p) {
+    chunk_attn_kernel(const __grid_constant__ P p) {
+  constexpr bool kWaves = std::is_same<P, AttnParamsWaves>::value;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -389,6 +412,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + SM_MISC + 4);
   volatile int* comb_flag = reinterpret_cast<volatile int*>(smem + SM_MISC + 8);  // [Q_TILES]
   int* prefix = reinterpret_cast<int*>(smem + SM_PREFIX);
+  unsigned* tb = reinterpret_cast<unsigned*>(smem + SM_TB);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -429,6 +453,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tmem_relinquish();
   }
   for (int g = tid; g < p.n_qg; g += NTHREADS) prefix[g + 1] = unit_tile_count(p.sched, g);
+  if constexpr (kWaves) {
+    for (int c = tid; c <= p.G; c += NTHREADS) tb[c] = p.tb[c];
+  }
   // rotary view: the call's table rows copied to shared memory when they fit
   RopeTables rope = p.rope;
   if (p.stage_ok) {
@@ -465,8 +492,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const Cursor cstart = {0, p.tb[blockIdx.x]};
-  const unsigned cend = p.tb[blockIdx.x + 1];
+  Cursor cstart;
+  unsigned cend;
+  if constexpr (kWaves) {
+    cstart = {0, p.tb[blockIdx.x]};
+    cend = p.tb[blockIdx.x + 1];
+  } else {
+    cstart = {0, cta_start(blockIdx.x, p.W, p.G)};
+    cend = cta_start(blockIdx.x + 1, p.W, p.G);
+  }
 
   if (warp < WARP_SOFT) {
   regs_dec<REGS_CTRL>();
@@ -713,14 +747,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       row_ranges(p.sched, s_eff, a0, a1, b0, b1);
       float m_run = -INFINITY, l_run = 0.f;
       for (int i = 0; i < sg.n; ++i, ++tn) {
-        if (!mbar_wait(&bar[B_S_FULL + q], tn & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
+        // the tile's visible-column ranges, worked out before its scores are ready
         const KTile kt = ktile(p, seg_tile(sg, i));
         const int la = max(0, min(TILE_N, a0 - kt.vbase));
         const int ha = max(0, min(kt.nvalid, a1 - kt.vbase));
         const int lb = max(0, min(TILE_N, b0 - kt.vbase));
         const int hb = max(0, min(kt.nvalid, b1 - kt.vbase));
         const bool full = (la == 0 && ha == TILE_N);
+        if (!mbar_wait(&bar[B_S_FULL + q], tn & 1, abort_flag, p.status)) { ok = false; break; }
+        tc_fence_after();
         uint32_t v0[32], v1[32], v2[32], v3[32];
         tmem_ld32(tS, v0);
         tmem_ld32(tS + 32, v1);
@@ -818,12 +853,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // row as float2.
         constexpr int ROWS = Q_TILES * TILE_M;
         const int row_l = q * TILE_M + r;
-        const int c_first = cta_of(p, sg.u0);
-        const int c_last = cta_of(p, sg.u1 - 1);
+        const int c_first = kWaves ? cta_of(tb, p.G, sg.u0) : cta_of(sg.u0, p.W, p.G);
+        const int c_last = kWaves ? cta_of(tb, p.G, sg.u1 - 1) : cta_of(sg.u1 - 1, p.W, p.G);
         const int np = c_last - c_first + 1;
         // slot of the piece held by CTA c: its first segment (slot 2c) unless the
         // unit began before c's range, which only the first piece's CTA can see
-        const int slot0 = 2 * c_first + (p.tb[c_first] == sg.u0 ? 0 : 1);
+        const unsigned start_first = kWaves ? tb[c_first] : cta_start(c_first, p.W, p.G);
+        const int slot0 = 2 * c_first + (start_first == sg.u0 ? 0 : 1);
         const int me = static_cast<int>(blockIdx.x) - c_first;  // piece index
         auto slot_of = [&](int k) { return k == 0 ? slot0 : 2 * (c_first + k); };
         int* counter = p.counters + (static_cast<size_t>(sg.bh) * p.n_qg + sg.qg) * Q_TILES + q;
@@ -967,22 +1003,26 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
+template <class P>
+static cudaError_t prepare_kernel() {
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
     // the warpgroup register split assumes exactly LAUNCH_REGS registers per thread
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_attn_kernel);
+    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_attn_kernel<P>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(chunk_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunk_attn_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  AttnParams p;
+  return cudaSuccess;
+}
+
+static void fill_params(AttnParams& p, const AttnLaunch& a) {
   p.tm_q = a.tm_q;
   p.tm_k = a.tm_k;
   p.tm_v = a.tm_v;
@@ -1004,11 +1044,28 @@ cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
   p.stage_ok = a.stage_ok;
   p.stage_t0 = a.stage_t0;
   p.stage_nt = a.stage_nt;
+  p.W = static_cast<unsigned>(a.W);
   p.G = a.grid;
-  p.waves = a.waves;
-  for (int c = 0; c <= a.grid; ++c) p.tb[c] = a.tb[c];
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));
-  chunk_attn_kernel<<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+}
+
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
+  // the plain split computes c * W / G in 32 bits; past that the ranges go explicitly
+  if (a.waves > 0 || a.W * (a.grid + 1LL) >= (1LL << 31)) {
+    cudaError_t e = prepare_kernel<AttnParamsWaves>();
+    if (e != cudaSuccess) return e;
+    AttnParamsWaves p;
+    fill_params(p, a);
+    p.waves = a.waves;
+    for (int c = 0; c <= a.grid; ++c) p.tb[c] = a.tb[c];
+    chunk_attn_kernel<AttnParamsWaves><<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+  } else {
+    cudaError_t e = prepare_kernel<AttnParams>();
+    if (e != cudaSuccess) return e;
+    AttnParams p;
+    fill_params(p, a);
+    chunk_attn_kernel<AttnParams><<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+  }
   return cudaGetLastError();
 }
 

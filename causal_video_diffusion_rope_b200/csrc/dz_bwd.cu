@@ -25,7 +25,7 @@
 // thread writes its bf16 operands over its own fp32 columns, so a half's operand
 // occupies columns [0, 16) and [32, 48) of its region (see mma_tmem_a64).  The rotation back (R^T) and the 1/sqrt(128) are applied to the fp32
 // accumulators in the epilogue.
-#include "dz_internal.cuh"
+#include "dz_ops.cuh"
 #include "dz_ptx.cuh"
 
 namespace dz {

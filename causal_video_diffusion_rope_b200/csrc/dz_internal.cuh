@@ -15,7 +15,7 @@ constexpr int TILE_N = 128;        // keys per K/V tile
 constexpr int Q_TILES = 2;         // Q tiles per CTA (ping-pong between two softmax groups)
 constexpr int Q_GROUP = TILE_M * Q_TILES;  // query rows per work unit
 constexpr int MAX_Q_GROUPS = 512;  // per (batch, head); bounds the per-CTA prefix table
-constexpr int MAX_GRID = 512;      // CTAs of one attention launch (the schedule is a kernel parameter)
+constexpr int MAX_GRID = 256;      // CTAs of one attention launch (the schedule is a kernel parameter)
 
 // Rotary tables: (cos, sin) as float2 for every (axis position, pair of that axis).
 struct RopeTables {
@@ -178,6 +178,8 @@ struct AttnLaunch {
   // Schedule over `grid` CTAs: `waves` rounds of whole units dealt round-robin (CTA c
   // takes unit c + k * grid of the head-major order), then CTA c takes the flattened
   // key tiles [tb[c], tb[c + 1]) of the remaining units, splitting units between CTAs.
+  // With waves == 0, tb[c] = c * W / grid (W = all units' key tiles).
+  long long W;
   int grid;
   int waves;
   unsigned tb[MAX_GRID + 1];
@@ -199,38 +201,6 @@ constexpr int UNIT_SWITCH_TILES = 2;
 constexpr int ROPE_STAGE_MAX = 1280;
 
 cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream);
-
-// Fused QKV projection + rotation (+ cache append); see dz_qkv.cu.
-struct QkvLaunch {
-  CUtensorMap tm_x, tm_w;  // x [M][K], w [3*H*128][K], bf16, 64 x 256 boxes, SW128
-  void *q, *k, *v;         // [M][H][128]
-  void *ck, *cv;           // cache or null
-  int cache_cap, cache_row0;
-  int M, S, H, K;
-  RopeTables rope;
-  ChunkGeom geom;
-  int first_chunk;
-  int stage_ok, stage_t0, stage_nt;  // rotary rows staged in shared memory (see AttnLaunch)
-  int* status;
-  int num_sms;
-};
-// Capacity (float2 entries) of the projection kernel's shared-memory rotary table.
-constexpr int QKV_ROPE_STAGE_MAX = 4096;
-cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream);
-
-// Backward of the prefill / teacher-forcing attention; see dz_bwd.cu.
-struct BwdLaunch {
-  CUtensorMap tm_q, tm_k, tm_v, tm_do;  // rotated q, rotated k, v, dO (4-D, 128-row boxes)
-  const void *out, *dout;               // bf16 [B][S][H][128]
-  const float* lse;                     // [B][H][S] from the forward (log2 domain)
-  float* dd;                            // workspace [B][H][S]: rowsum(dO * O)
-  void *dq, *dk, *dv;                   // bf16 [B][S][H][128]
-  RopeTables rope;
-  ChunkGeom geom;
-  int mode, N, S, B, H;
-  int* status;
-};
-cudaError_t launch_backward(const BwdLaunch& a, cudaStream_t stream);
 
 // Workspace (in floats) one partial-result slot needs: Q_TILES * TILE_M rows of
 // HEAD_DIM accumulators plus (m, l) per row.

@@ -11,16 +11,19 @@
 // ("DreamZero (WAM) 模型架构", §2.3 block diagram: RMSNorm, modulation, causal
 // self-attention with RoPE on the latent sequence).
 //
-// One persistent CTA per SM walks output tiles of 256 tokens x 256 features
-// (two heads), n-tile major so that the CTAs working at one time share the
-// same weight tile through L2.  A tile is two 128-row halves that share each
-// weight slice, so every byte brought to the SM feeds twice the products of a
-// 128 x 256 tile.  Warp 0 issues TMA loads of 64-wide K slices into a 3-stage
-// ring, warp 1 allocates TMEM and issues tcgen05.mma (M=128, N=256, K=16, both
-// operands K-major SW128 in shared memory; two per K step, one per half) into
-// two 256-column TMEM accumulators, and warps 2-9 (one per TMEM lane quarter
-// and half) drain them (rotation, bf16 rounding, stores).
-#include "dz_internal.cuh"
+// One persistent CTA per SM walks output tiles of 256 tokens x BN features,
+// n-tile major so that the CTAs working at one time share the same weight tile
+// through L2.  BN (a multiple of 16, at most 256) is chosen per call so that the
+// tiles fill the SMs in as few waves as possible (for one 464-token chunk of the
+// 40-head DiT, BN = 208 gives 2 x 74 = 148 tiles, one per SM).  A tile is two
+// 128-row halves that share each weight slice, so every byte brought to the SM
+// feeds twice the products of a 128 x BN tile.  Warp 0 issues TMA loads of
+// 64-wide K slices into a 3-stage ring, warp 1 allocates TMEM and issues
+// tcgen05.mma (M=128, N=BN, K=16, both operands K-major SW128 in shared memory;
+// two per K step, one per half) into two TMEM accumulators, and warps 2-9 (one
+// per TMEM lane quarter and half) drain them 16 features at a time (rotation,
+// bf16 rounding, stores).
+#include "dz_ops.cuh"
 #include "dz_ptx.cuh"
 
 namespace dz {
@@ -28,6 +31,7 @@ namespace dz {
 namespace {
 
 constexpr int QBM = 256, QBN = 256, QBK = 64, QSTAGES = 3;
+constexpr int QPREFETCH = 8;             // weight K slices requested into L2 ahead of their load
 constexpr int QHALF = 128;               // rows per MMA (one TMEM lane each)
 constexpr int QTHREADS = 320;            // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
 constexpr int QA_BYTES = QBM * QBK * 2;  // 32 KiB
@@ -55,6 +59,7 @@ struct __align__(64) QkvParams {
   __nv_bfloat16 *ck, *cv;  // cache (null: no append)
   int cache_cap, cache_row0;
   int M, S, H, K, N;
+  int bn;  // features per tile
   int m_tiles, n_tiles;
   RopeTables rope;
   ChunkGeom geom;
@@ -63,11 +68,20 @@ struct __align__(64) QkvParams {
   int* status;
 };
 
-// 16 B stores of 32 bf16 values (a 64-byte row piece).
-__device__ __forceinline__ void store_piece(__nv_bfloat16* dst, const uint32_t (&pk)[16]) {
+// Requests a 2-D tile into L2 (no shared memory, no completion): the later TMA
+// load of the same tile then finds it there.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1)
+               : "memory");
+}
+
+// 16 B stores of 16 bf16 values (a 32-byte row piece).
+__device__ __forceinline__ void store_piece(__nv_bfloat16* dst, const uint32_t (&pk)[8]) {
   uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) d[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+  d[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  d[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
 
@@ -113,14 +127,18 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
         const int nt = tile / p.m_tiles, mt = tile - nt * p.m_tiles;
+        // the weight slices stream from DRAM: ask for them well before the ring has room
+        for (int j = QSTAGES; j < QPREFETCH && j < KB; ++j)
+          tma_prefetch_l2_2d(&p.tm_w, j * QBK, nt * p.bn);
         for (int kb = 0; kb < KB; ++kb, ++it) {
+          if (kb + QPREFETCH < KB) tma_prefetch_l2_2d(&p.tm_w, (kb + QPREFETCH) * QBK, nt * p.bn);
           const int st = it % QSTAGES;
           const uint32_t ph = (it / QSTAGES) & 1;
           if (!mbar_wait(&bar[QB_EMPTY + st], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint8_t* sa = smem + st * QSTAGE_BYTES;
-          mbar_expect_tx(&bar[QB_FULL + st], QSTAGE_BYTES);
+          mbar_expect_tx(&bar[QB_FULL + st], QA_BYTES + p.bn * QBK * 2);
           tma_load_2d(sa, &p.tm_x, &bar[QB_FULL + st], kb * QBK, mt * QBM);
-          tma_load_2d(sa + QA_BYTES, &p.tm_w, &bar[QB_FULL + st], kb * QBK, nt * QBN);
+          tma_load_2d(sa + QA_BYTES, &p.tm_w, &bar[QB_FULL + st], kb * QBK, nt * p.bn);
         }
       }
       // every issued copy has landed before the CTA exits
@@ -131,7 +149,7 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
   } else if (warp == 1) {
     // ---------------- tcgen05 issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(QHALF, QBN, false);
+      const uint32_t idesc = idesc_bf16(QHALF, p.bn, false);
       const uint32_t base_lo = desc_lo(smem_u32(smem), 16);
       uint32_t it = 0;
       int lt = 0;
@@ -199,58 +217,57 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
       const int s = valid ? m - bb * p.S : 0;
       int t = 0, hh = 0, w = 0;
       token_pos(p.geom, s, p.first_chunk, t, hh, w);
-      // 32-column pieces in the order (dims 0-31 of both heads, dims 32-63 of both, ...)
-      // so that each set of 16 (cos, sin) entries is read once for the two heads
+      // 16-feature pieces: each lies inside one head (16 divides 128 and BN); piece
+      // c + 1 is read from TMEM while piece c is turned and stored
+      int pieces = p.bn / 16;
+      if (nt * p.bn + pieces * 16 > p.N) pieces = (p.N - nt * p.bn) / 16;
+      uint32_t v[16], vn[16];
+      tmem_ld16(tmem + lane_addr + half * QBN, v);
+      tmem_wait_ld();
 #pragma unroll 1
-      for (int dq = 0; dq < HEAD_DIM / 32; ++dq) {
-        float2 cs[16];
-        if (nt * QBN < 2 * HD) {  // the tile holds q or k features
+      for (int c = 0; c < pieces; ++c) {
+        const int n = nt * p.bn + c * 16;  // feature of column 0 of this piece
+        if (c + 1 < pieces) tmem_ld16(tmem + lane_addr + half * QBN + (c + 1) * 16, vn);
+        const int sec = n / HD;  // 0 q, 1 k, 2 v
+        const int rem = n - sec * HD;
+        const int head = rem / HEAD_DIM, d0 = rem - head * HEAD_DIM;
+        float2 cs[8];
+        if (sec < 2) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            cs[i] = rope.tab[rope_index(rope, dq * 16 + i, t, hh, w)];
+          for (int i = 0; i < 8; ++i) cs[i] = rope.tab[rope_index(rope, d0 / 2 + i, t, hh, w)];
         }
-#pragma unroll 1
-        for (int hp = 0; hp < QBN / HEAD_DIM; ++hp) {
-          const int c = hp * (HEAD_DIM / 32) + dq;
-          uint32_t v[32];
-          tmem_ld32(tmem + lane_addr + half * QBN + c * 32, v);
-          tmem_wait_ld();
-          if (dq == HEAD_DIM / 32 - 1 && hp == QBN / HEAD_DIM - 1) {
-            tc_fence_before();
-            mbar_arrive(&bar[QB_ACC_EMPTY]);
-          }
-          const int n = nt * QBN + c * 32;  // feature of column 0 of this piece
-          if (n >= p.N) continue;
-          const int sec = n / HD;  // 0 q, 1 k, 2 v
-          const int rem = n - sec * HD;
-          const int head = rem / HEAD_DIM, d0 = rem - head * HEAD_DIM;
-          uint32_t pk[16];
-          if (sec < 2) {
+        uint32_t pk[8];
+        if (sec < 2) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
-              const float y0 = __fmaf_rn(x0, cs[i].x, -__fmul_rn(x1, cs[i].y));
-              const float y1 = __fmaf_rn(x0, cs[i].y, __fmul_rn(x1, cs[i].x));
-              pk[i] = pack_bf16x2(y0, y1);
-            }
-          } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-              pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+          for (int i = 0; i < 8; ++i) {
+            const float x0 = __uint_as_float(v[2 * i]), x1 = __uint_as_float(v[2 * i + 1]);
+            const float y0 = __fmaf_rn(x0, cs[i].x, -__fmul_rn(x1, cs[i].y));
+            const float y1 = __fmaf_rn(x0, cs[i].y, __fmul_rn(x1, cs[i].x));
+            pk[i] = pack_bf16x2(y0, y1);
           }
-          if (valid) {
-            __nv_bfloat16* dst = (sec == 0 ? p.q : (sec == 1 ? p.k : p.v)) +
-                                 (static_cast<size_t>(m) * p.H + head) * HEAD_DIM + d0;
-            store_piece(dst, pk);
-            if (sec > 0 && p.ck) {
-              __nv_bfloat16* cdst = (sec == 1 ? p.ck : p.cv) +
-                                    ((static_cast<size_t>(bb) * p.cache_cap + p.cache_row0 + s) * p.H +
-                                     head) * HEAD_DIM + d0;
-              store_piece(cdst, pk);
-            }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+        }
+        if (valid) {
+          __nv_bfloat16* dst = (sec == 0 ? p.q : (sec == 1 ? p.k : p.v)) +
+                               (static_cast<size_t>(m) * p.H + head) * HEAD_DIM + d0;
+          store_piece(dst, pk);
+          if (sec > 0 && p.ck) {
+            __nv_bfloat16* cdst = (sec == 1 ? p.ck : p.cv) +
+                                  ((static_cast<size_t>(bb) * p.cache_cap + p.cache_row0 + s) * p.H +
+                                   head) * HEAD_DIM + d0;
+            store_piece(cdst, pk);
           }
         }
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = vn[i];
       }
+      // this thread's accumulator loads are complete: the MMA warp may reuse them
+      tc_fence_before();
+      mbar_arrive(&bar[QB_ACC_EMPTY]);
     }
   }
 
@@ -263,7 +280,25 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
   }
 }
 
+int qkv_tile_n(long long M, long long N, int num_sms) {
+  // least work for the busiest SM: waves x (BN + a fixed 32 for the token slice each
+  // K step also loads), the larger BN on a tie
+  const long long m_tiles = (M + QBM - 1) / QBM;
+  int best = QBN;
+  long long best_cost = -1;
+  for (int bn = QBN; bn >= 64; bn -= 16) {
+    const long long tiles = m_tiles * ((N + bn - 1) / bn);
+    const long long cost = (tiles + num_sms - 1) / num_sms * (bn + 32);
+    if (best_cost < 0 || cost < best_cost) {
+      best = bn;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream) {
+  if (a.bn < 16 || a.bn > QBN || a.bn % 16 != 0) return cudaErrorInvalidValue;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -288,8 +323,9 @@ cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream) {
   p.H = a.H;
   p.K = a.K;
   p.N = 3 * a.H * HEAD_DIM;
+  p.bn = a.bn;
   p.m_tiles = (a.M + QBM - 1) / QBM;
-  p.n_tiles = (p.N + QBN - 1) / QBN;
+  p.n_tiles = (p.N + p.bn - 1) / p.bn;
   p.rope = a.rope;
   p.geom = a.geom;
   p.first_chunk = a.first_chunk;

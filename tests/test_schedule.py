@@ -2,9 +2,10 @@
 dz_test_plan_schedule: for a call whose (batch, head) pairs each have query groups
 with the given key-tile counts, CTA c first takes whole units c + k * grid for
 k < waves (head-major order), then the flattened key tiles [tb[c], tb[c + 1]) of
-the remaining units.  Checked without a GPU: every key tile of every unit is
-covered exactly once, the ranges are ordered, the whole-unit waves leave a tail
-of at least half a wave, and the estimated work per CTA is balanced.  The tile
+the remaining units; units of equal size get no waves and tb[c] = c * W / grid.
+Checked without a GPU: every key tile of every unit is covered exactly once, the
+ranges are ordered, the whole-unit waves leave a tail of at least half a wave, and
+the estimated work per CTA is balanced.  The tile
 counts of the real workloads are counted here from the oracle's visibility matrix."""
 import ctypes
 
@@ -14,7 +15,7 @@ import pytest
 from causal_video_diffusion_rope_b200 import build, synth
 from oracle import dz_oracle as O
 
-MAX_GRID = 512
+MAX_GRID = 256
 SWITCH = 2  # estimated start-up cost of a whole unit, in key tiles (as in the planner)
 
 
@@ -109,10 +110,29 @@ def test_teacher_forcing_uses_whole_unit_waves(lib):
 
 
 def test_decode_few_units_one_per_cta(lib):
-    # 8 units of 3 tiles on 148 SMs: one CTA per unit, no tail
+    # 8 equal units of 3 tiles on 148 SMs: one CTA per unit through the plain split
     g, waves, tb = plan(lib, [3, 3], 4, 148)
-    assert g == 8 and waves == 1 and tb == [24] * 9  # W = 4 pairs x 2 groups x 3 tiles
+    assert g == 8 and waves == 0 and tb == [3 * c for c in range(9)]
     check([3, 3], 4, 148, g, waves, tb)
+
+
+def test_ragged_few_units_one_per_cta(lib):
+    # 8 units of 3 or 4 tiles: one whole-unit wave, no tail
+    g, waves, tb = plan(lib, [3, 4], 4, 148)
+    assert g == 8 and waves == 1 and tb == [28] * 9  # W = 4 pairs x 7 tiles
+    check([3, 4], 4, 148, g, waves, tb)
+
+
+@pytest.mark.parametrize("wi", range(len(synth.WORKLOADS)))
+def test_equal_units_never_use_waves(lib, wi):
+    # decode and cross-attention units all see the same key tiles: the plain split
+    w = synth.WORKLOADS[wi]
+    tiles = group_tiles(w)
+    if len(set(tiles)) != 1:
+        pytest.skip("ragged units")
+    g, waves, tb = plan(lib, tiles, w.layout.batch * w.heads, 148)
+    W = sum(tiles) * w.layout.batch * w.heads
+    assert waves == 0 and tb == [c * W // g for c in range(g + 1)]
 
 
 @pytest.mark.parametrize("seed", range(6))
