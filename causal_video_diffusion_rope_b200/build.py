@@ -1,9 +1,13 @@
 """Build libdz.so (the C-ABI library) in-tree for sm_100a with nvcc.
 
-Also builds libdz_test.so from the same sources for the device-timeout tests:
-every bounded device wait gives up after 20 ms instead of 2 s, and the library
-exports one extra call, dz_test_fill_split_counters, that presets the split
-counters so that a merge's wait can never complete.  Nothing but the tests loads it.
+Also builds libdz_test.so from the same sources for the tests: every bounded
+device wait gives up after 20 ms instead of 2 s; every kernel checks its global
+indexes against the extents of their buffers (DZ_DEBUG_BOUNDS: a failed check skips
+the access and records DZ_ERR_BOUNDS in the status word); and the library exports
+test-only calls: dz_test_fill_split_counters (presets the split counters so that a
+merge's wait can never complete), dz_test_shrink_out (understates the attention
+output's extent), dz_test_bounds_faults (index faults counted on the host) and
+dz_test_plan_schedule (the attention work split).  Nothing but the tests loads it.
 
 Usage: python -m causal_video_diffusion_rope_b200.build [--verbose-ptxas]
 """
@@ -19,7 +23,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdz.so")
 TEST_LIB = os.path.join(HERE, "libdz_test.so")
-TEST_DEFINES = ["-DDZ_TEST_HOOKS", "-DDZ_WAIT_NS=20000000ull"]
+TEST_DEFINES = ["-DDZ_TEST_HOOKS", "-DDZ_DEBUG_BOUNDS", "-DDZ_WAIT_NS=20000000ull"]
 SOURCES = ["dz_api.cu", "dz_kernels.cu", "dz_attn.cu", "dz_qkv.cu", "dz_bwd.cu"]
 HEADERS = ["dz_internal.cuh", "dz_ops.cuh", "dz_ptx.cuh"]
 

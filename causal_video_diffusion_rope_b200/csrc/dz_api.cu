@@ -98,6 +98,7 @@ dz::RopeTables tables_of(const dz_attn* a) {
   r.pt = a->desc.rope_pairs_t;
   r.ph = a->desc.rope_pairs_h;
   r.pw = a->desc.rope_pairs_w;
+  r.n = a->off_w + a->desc.max_pos_w * a->desc.rope_pairs_w;
   return r;
 }
 
@@ -118,7 +119,21 @@ dz_status check_positions(const dz_attn* a, const dz::ChunkGeom& g, long long fi
 // merging piece's wait for the others' publications can never complete, so the
 // bounded wait runs out and the call reports DZ_ERR_TIMEOUT.
 int g_test_counter_fill = 0;
+// Elements taken off the attention output's extent (dz_test_shrink_out), and the index
+// faults of the bounds-checked kernels counted on the host (dz_test_bounds_faults).
+long long g_test_out_shrink = 0;
+long long g_test_bounds_faults = 0;
 #endif
+
+// Status of a nonzero device status word: an index fault of the bounds-checked build
+// takes precedence over a wait that ran out (which it may have caused).
+dz_status status_of_word(int word) {
+#ifdef DZ_TEST_HOOKS
+  if (word & dz::DZ_DEV_BOUNDS) ++g_test_bounds_faults;
+#endif
+  return (word & dz::DZ_DEV_BOUNDS) ? DZ_ERR_BOUNDS : DZ_ERR_TIMEOUT;
+}
+
 
 }  // namespace
 
@@ -210,6 +225,17 @@ extern "C" {
 #ifdef DZ_TEST_HOOKS
 void dz_test_fill_split_counters(int32_t value) { g_test_counter_fill = value; }
 
+// Takes n elements off the output extent the next attention launches are given, so
+// that the bounds-checked build's store checks fail for the last n elements.
+void dz_test_shrink_out(int64_t n) { g_test_out_shrink = n; }
+
+// Index faults seen by dz_attn_sync_status or dz_attn_destroy since the last call.
+int64_t dz_test_bounds_faults(void) {
+  const long long n = g_test_bounds_faults;
+  g_test_bounds_faults = 0;
+  return n;
+}
+
 // The work split of an attention call for `bh_count` (batch, head) pairs whose query
 // groups have tiles[0 .. n_qg) key tiles each, over at most num_sms CTAs: writes the
 // grid, the number of whole-unit waves and the tail ranges (grid + 1 entries of tb).
@@ -234,6 +260,7 @@ const char* dz_status_string(dz_status s) {
     case DZ_ERR_CUDA: return "CUDA error";
     case DZ_ERR_UNSUPPORTED: return "unsupported";
     case DZ_ERR_TIMEOUT: return "device wait timed out";
+    case DZ_ERR_BOUNDS: return "device index check failed";
   }
   return "unknown status";
 }
@@ -333,6 +360,13 @@ dz_status dz_attn_create(dz_attn_t* out, const dz_attn_desc* d) {
 dz_status dz_attn_destroy(dz_attn_t a) {
   if (!a) return DZ_ERR_INVALID_ARG;
   cudaError_t e = cudaDeviceSynchronize();
+#ifdef DZ_TEST_HOOKS
+  // an index fault that no status read reported is still counted
+  int word = 0;
+  if (e == cudaSuccess && cudaMemcpy(&word, a->status, sizeof(int), cudaMemcpyDeviceToHost) ==
+                              cudaSuccess && (word & dz::DZ_DEV_BOUNDS))
+    ++g_test_bounds_faults;
+#endif
   cudaFree(a->rope_tab);
   cudaFree(a->ws);
   cudaFree(a->counters);
@@ -356,7 +390,7 @@ dz_status dz_rope3d(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
   st = check_positions(a, g, first_chunk, first_chunk + (S - 1) / g.L);
   if (st != DZ_OK) return st;
   return cuda_status(dz::launch_rope3d(x, y, B, S, a->desc.num_heads, g, first_chunk,
-                                       tables_of(a), static_cast<cudaStream_t>(stream)),
+                                       tables_of(a), a->status, static_cast<cudaStream_t>(stream)),
                      "rope3d launch");
 }
 
@@ -466,8 +500,8 @@ static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const v
     const int period = l->mode == DZ_MODE_TEACHER_FORCING ? static_cast<int>(L * l->num_chunks) : 0;
     const int first = l->mode == DZ_MODE_DECODE ? l->num_chunks : 0;
     st = cuda_status(dz::launch_rope3d(q, qr, l->batch, static_cast<int>(Sq), H, g, first,
-                                       tables_of(a), static_cast<cudaStream_t>(stream), k, kr,
-                                       period),
+                                       tables_of(a), a->status, static_cast<cudaStream_t>(stream),
+                                       k, kr, period),
                      "pre-rotation launch");
     if (st != DZ_OK) return st;
     q_att = qr;
@@ -480,6 +514,12 @@ static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const v
   p.ws = a->ws;
   p.counters = a->counters;
   p.status = a->status;
+  p.out_elems = static_cast<long long>(l->batch) * Sq * H * dz::HEAD_DIM;
+  p.ws_slots = 2 * a->num_sms;
+  p.n_counters = static_cast<long long>(a->n_counters);
+#ifdef DZ_TEST_HOOKS
+  p.out_elems -= g_test_out_shrink;
+#endif
 
   st = make_map(a, &p.tm_q, q_att, l->batch, static_cast<int>(Sq), static_cast<int>(Sq), H);
   if (st == DZ_OK) st = make_map(a, &p.tm_k, k_att, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
@@ -527,7 +567,7 @@ dz_status dz_kvcache_append(dz_attn_t a, dz_kvcache* c, const void* k, const voi
   if (static_cast<long long>(c->len_tokens) + c->chunk_len > c->capacity_tokens)
     return DZ_ERR_CAPACITY;
   cudaError_t e = dz::launch_kv_copy(k, v, c->k, c->v, c->batch, c->chunk_len, a->desc.num_heads,
-                                     c->capacity_tokens, c->len_tokens,
+                                     c->capacity_tokens, c->len_tokens, a->status,
                                      static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return DZ_ERR_CUDA;
   c->len_tokens += c->chunk_len;
@@ -546,7 +586,7 @@ dz_status dz_kvcache_replace(dz_attn_t a, dz_kvcache* c, int32_t chunk_index, co
     return DZ_ERR_ALIGNMENT;
   return cuda_status(dz::launch_kv_copy(k, v, c->k, c->v, c->batch, c->chunk_len,
                                         a->desc.num_heads, c->capacity_tokens,
-                                        chunk_index * c->chunk_len,
+                                        chunk_index * c->chunk_len, a->status,
                                         static_cast<cudaStream_t>(stream)));
 }
 
@@ -582,6 +622,7 @@ dz_status dz_qkv_rope(dz_attn_t a, const void* x, const void* w, int32_t B, int3
     p.cv = cache->v;
     p.cache_cap = cache->capacity_tokens;
     p.cache_row0 = cache->len_tokens;
+    p.cache_batch = cache->batch;
   }
   // x as [M][d_model] with 64 x 256 boxes, w as [N][d_model] with 64 x bn boxes
   p.bn = dz::qkv_tile_n(M, N, a->num_sms);
@@ -654,7 +695,7 @@ dz_status dz_chunk_attn_backward(dz_attn_t a, const void* q, const void* k, cons
   __nv_bfloat16* kr = qr + elems;
   const int period = l->mode == DZ_MODE_TEACHER_FORCING ? g.L * l->num_chunks : 0;
   st = cuda_status(dz::launch_rope3d(q, qr, l->batch, static_cast<int>(S), H, g, 0, tables_of(a),
-                                     static_cast<cudaStream_t>(stream), k, kr, period),
+                                     a->status, static_cast<cudaStream_t>(stream), k, kr, period),
                    "backward rotation launch");
   if (st != DZ_OK) return st;
   dz::BwdLaunch p;
@@ -696,7 +737,7 @@ dz_status dz_attn_sync_status(dz_attn_t a, void* stream) {
         cudaMemset(a->counters, 0, a->n_counters * sizeof(int)) != cudaSuccess ||
         cudaDeviceSynchronize() != cudaSuccess)
       return DZ_ERR_CUDA;
-    return DZ_ERR_TIMEOUT;
+    return status_of_word(word);
   }
   return DZ_OK;
 }
@@ -886,5 +927,5 @@ static dz_status noalloc_sync_status(void* stream) {
       cudaMemset(counters, 0, NOALLOC_COUNTERS * sizeof(int)) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess)
     return DZ_ERR_CUDA;
-  return DZ_ERR_TIMEOUT;
+  return status_of_word(word);
 }

@@ -107,6 +107,9 @@ struct __align__(64) AttnParams {
   float* ws;
   int* counters;
   int* status;
+  long long out_elems;   // B * Sq * H * 128 (bounds-checked build)
+  int ws_slots;          // partial-result slots of ws
+  long long n_counters;  // split counters
   RopeTables rope;
   ChunkGeom geom;
   SchedGeom sched;
@@ -271,7 +274,7 @@ __device__ __forceinline__ void seq_pos(const AttnParams& p, int s, int& t, int&
 // values of four chunks are loaded before their shared-memory read-modify-write
 // so that the loads overlap.  `rt.tab` may point to shared or global memory.
 __device__ __forceinline__ void rotate_tile_row(uint8_t* tile, int r, const RopeTables& rt, int t,
-                                                int h, int w) {
+                                                int h, int w, int* status) {
   uint8_t* row = tile + r * 128;
 #pragma unroll
   for (int b4 = 0; b4 < 4; ++b4) {
@@ -280,7 +283,7 @@ __device__ __forceinline__ void rotate_tile_row(uint8_t* tile, int r, const Rope
     for (int k = 0; k < 4; ++k) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        cs[4 * k + i] = rt.tab[rope_index(rt, (b4 * 4 + k) * 4 + i, t, h, w)];
+        cs[4 * k + i] = rt.tab[rope_index_checked(rt, (b4 * 4 + k) * 4 + i, t, h, w, status)];
     }
     uint4 v[4];
 #pragma unroll
@@ -464,12 +467,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float2* gt = p.rope.tab + p.rope.off_t + p.stage_t0 * p.rope.pt;
     const float2* gh = p.rope.tab + p.rope.off_h;
     const float2* gw = p.rope.tab + p.rope.off_w;
-    for (int i = tid; i < nt + nh + nw; i += NTHREADS)
-      st_tab[i] = i < nt ? gt[i] : (i < nt + nh ? gh[i - nt] : gw[i - nt - nh]);
+    for (int i = tid; i < nt + nh + nw; i += NTHREADS) {
+      const long long gi = i < nt ? p.rope.off_t + static_cast<long long>(p.stage_t0) * p.rope.pt + i
+                                  : (i < nt + nh ? p.rope.off_h + i - nt : p.rope.off_w + i - nt - nh);
+      if (in_bounds(gi, p.rope.n, p.status))
+        st_tab[i] = i < nt ? gt[i] : (i < nt + nh ? gh[i - nt] : gw[i - nt - nh]);
+    }
     rope.tab = st_tab;
     rope.off_t = -p.stage_t0 * p.rope.pt;
     rope.off_h = nt;
     rope.off_w = nt + nh;
+    rope.n = nt + nh + nw;
   }
   __syncthreads();
   if (warp == 0) {  // inclusive scan of the counts -> prefix[0..n_qg]
@@ -679,7 +687,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         rotate_tile_row_split<22, 21, 21>(smem_u32(tile), r, st_base + 8 * ((t - p.stage_t0) * 22),
                                           st_h + 8 * (h * 21), st_w + 8 * (w * 21));
       } else {
-        rotate_tile_row(tile, r, rope, t, h, w);
+        rotate_tile_row(tile, r, rope, t, h, w, p.status);
       }
     };
     Cursor pos = cstart;
@@ -810,8 +818,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // bf16 out = O / l; each 32-column chunk goes through the warp's transpose
         // buffer so that global stores cover 64 contiguous bytes of 8 rows at a time
         const float inv_l = 1.f / l_run;
-        if (p.lse && s_tok < p.sched.Sq)
-          p.lse[(static_cast<size_t>(b) * p.H + h) * p.sched.Sq + s_tok] = m_run + __log2f(l_run);
+        if (p.lse && s_tok < p.sched.Sq) {
+          const long long li = (static_cast<long long>(b) * p.H + h) * p.sched.Sq + s_tok;
+          if (in_bounds(li, p.out_elems / HEAD_DIM, p.status)) p.lse[li] = m_run + __log2f(l_run);
+        }
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
@@ -836,10 +846,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int rr = task >> 2, piece = task & 3;
             const int s = row0 + rr;
             const uint4 val = *reinterpret_cast<const uint4*>(xp + rr * XPOSE_PITCH + piece * 16);
-            if (s < p.sched.Sq) {
-              __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + c * 32 + piece * 8;
-              *reinterpret_cast<uint4*>(dst) = val;
-            }
+            const long long oi = ((static_cast<long long>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + c * 32 + piece * 8;
+            if (s < p.sched.Sq && in_bounds(oi + 7, p.out_elems, p.status))
+              *reinterpret_cast<uint4*>(p.out + oi) = val;
           }
           __syncwarp();
         }
@@ -861,8 +870,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const unsigned start_first = kWaves ? tb[c_first] : cta_start(c_first, p.W, p.G);
         const int slot0 = 2 * c_first + (start_first == sg.u0 ? 0 : 1);
         const int me = static_cast<int>(blockIdx.x) - c_first;  // piece index
-        auto slot_of = [&](int k) { return k == 0 ? slot0 : 2 * (c_first + k); };
-        int* counter = p.counters + (static_cast<size_t>(sg.bh) * p.n_qg + sg.qg) * Q_TILES + q;
+        auto slot_of = [&](int k) {
+          const int sl = k == 0 ? slot0 : 2 * (c_first + k);
+          return in_bounds(sl, p.ws_slots, p.status) ? sl : 0;
+        };
+        long long ci = (static_cast<long long>(sg.bh) * p.n_qg + sg.qg) * Q_TILES + q;
+        if (!in_bounds(ci, p.n_counters, p.status)) ci = 0;
+        int* counter = p.counters + ci;
         if (gtid == 0) {
           const int old = atomicAdd(counter, 1);
           comb_flag[q] = ((old & 0xffff) == np - 1) ? 1 : 0;
@@ -952,8 +966,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_wait_st();
           }
           const float invL = 1.f / Lsum;
-          if (p.lse && s_tok < p.sched.Sq)
-            p.lse[(static_cast<size_t>(b) * p.H + h) * p.sched.Sq + s_tok] = M + __log2f(Lsum);
+          if (p.lse && s_tok < p.sched.Sq) {
+            const long long li = (static_cast<long long>(b) * p.H + h) * p.sched.Sq + s_tok;
+            if (in_bounds(li, p.out_elems / HEAD_DIM, p.status)) p.lse[li] = M + __log2f(Lsum);
+          }
 #pragma unroll 1
           for (int g = 0; g < 4; ++g) {  // 32 output columns per pass
             uint32_t v[32];
@@ -979,10 +995,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               const int rr = task >> 2, piece = task & 3;
               const int s = row0 + rr;
               const uint4 val = *reinterpret_cast<const uint4*>(xp + rr * XPOSE_PITCH + piece * 16);
-              if (s < p.sched.Sq) {
-                __nv_bfloat16* dst = p.out + ((static_cast<size_t>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + g * 32 + piece * 8;
-                *reinterpret_cast<uint4*>(dst) = val;
-              }
+              const long long oi = ((static_cast<long long>(b) * p.sched.Sq + s) * p.H + h) * HEAD_DIM + g * 32 + piece * 8;
+              if (s < p.sched.Sq && in_bounds(oi + 7, p.out_elems, p.status))
+                *reinterpret_cast<uint4*>(p.out + oi) = val;
             }
             __syncwarp();
           }
@@ -1033,6 +1048,9 @@ static void fill_params(AttnParams& p, const AttnLaunch& a) {
   p.ws = a.ws;
   p.counters = a.counters;
   p.status = a.status;
+  p.out_elems = a.out_elems;
+  p.ws_slots = a.ws_slots;
+  p.n_counters = a.n_counters;
   p.rope = a.rope;
   p.geom = a.geom;
   p.sched = a.sched;

@@ -127,11 +127,11 @@ __device__ __forceinline__ void bpos(const BwdParams& p, int s, int& t, int& h, 
 // -theta, scaled, rounded to bf16 and stored (16-byte stores).
 __device__ __forceinline__ void store_rotated_back(__nv_bfloat16* dst, const uint32_t (&v)[32],
                                                    const RopeTables& r, int c, int t, int h, int w,
-                                                   float scale) {
+                                                   float scale, int* status) {
   uint32_t pk[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float2 cs = __ldg(r.tab + rope_index(r, 16 * c + i, t, h, w));
+    const float2 cs = __ldg(r.tab + rope_index_checked(r, 16 * c + i, t, h, w, status));
     const float x0 = __uint_as_float(v[2 * i]) * scale, x1 = __uint_as_float(v[2 * i + 1]) * scale;
     const float y0 = __fmaf_rn(x0, cs.x, __fmul_rn(x1, cs.y));
     const float y1 = __fmaf_rn(x1, cs.x, -__fmul_rn(x0, cs.y));
@@ -289,7 +289,9 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
     const int s = q0 + r;
     const bool valid = s < p.S;
     const int s_eff = valid ? s : p.S - 1;
-    const size_t vec = static_cast<size_t>(bh) * p.S + s_eff;
+    size_t vec = static_cast<size_t>(bh) * p.S + s_eff;
+    if (!in_bounds(static_cast<long long>(vec), static_cast<long long>(p.B) * p.H * p.S, p.status))
+      vec = 0;
     const float lse2 = p.lse[vec];
     const float dsum = p.dd[vec];
     int a0, a1, b0, b1;
@@ -333,7 +335,10 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
       tc_fence_after();
       int t, hh, w;
       bpos(p, s_eff, t, hh, w);
-      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(b * p.S + s_eff) * p.H + h) * HEAD_DIM;
+      const long long dqi = (static_cast<long long>(b * p.S + s_eff) * p.H + h) * HEAD_DIM;
+      const bool dq_ok =
+          in_bounds(dqi + HEAD_DIM - 1, static_cast<long long>(p.B) * p.S * p.H * HEAD_DIM, p.status);
+      __nv_bfloat16* dst = p.dq + dqi;
 #pragma unroll 1
       for (int c = 2 * cg; c < 2 * cg + 2; ++c) {
         uint32_t v[32];
@@ -343,7 +348,7 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
 #pragma unroll
           for (int e = 0; e < 32; ++e) v[e] = 0u;
         }
-        if (valid) store_rotated_back(dst + 32 * c, v, p.rope, c, t, hh, w, p.scale);
+        if (valid && dq_ok) store_rotated_back(dst + 32 * c, v, p.rope, c, t, hh, w, p.scale, p.status);
       }
     }
   }
@@ -489,7 +494,9 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
       float* vb = sm_vec + (it & 1) * 2 * BT;
       {
         const int qq = q0 + (ct & (BT - 1));
-        vb[ct] = qq < p.S ? (ct < BT ? p.lse[vbase + qq] : p.dd[vbase + qq]) : 0.f;
+        const bool vin = qq < p.S && in_bounds(static_cast<long long>(vbase) + qq,
+                                               static_cast<long long>(p.B) * p.H * p.S, p.status);
+        vb[ct] = vin ? (ct < BT ? p.lse[vbase + qq] : p.dd[vbase + qq]) : 0.f;
       }
       named_bar_sync(1, BCOMPUTE);
       for (int hf = 0; hf < 2; ++hf) {
@@ -528,6 +535,8 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
     if (ok && mbar_wait(&bar[BB_ACC], 0, abort_flag, p.status)) {
       tc_fence_after();
       const size_t row = (static_cast<size_t>(b * p.S + j_eff) * p.H + h) * HEAD_DIM;
+      const bool row_ok = in_bounds(static_cast<long long>(row) + HEAD_DIM - 1,
+                                    static_cast<long long>(p.B) * p.S * p.H * HEAD_DIM, p.status);
       if (cg == 0) {  // dV
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
@@ -538,7 +547,7 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = 0u;
           }
-          if (valid) {
+          if (valid && row_ok) {
             uint4* d = reinterpret_cast<uint4*>(p.dv + row + 32 * c);
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -560,7 +569,8 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
 #pragma unroll
             for (int e = 0; e < 32; ++e) v[e] = 0u;
           }
-          if (valid) store_rotated_back(p.dk + row + 32 * c, v, p.rope, c, t, hh, w, p.scale);
+          if (valid && row_ok)
+            store_rotated_back(p.dk + row + 32 * c, v, p.rope, c, t, hh, w, p.scale, p.status);
         }
       }
     }

@@ -17,11 +17,32 @@ constexpr int Q_GROUP = TILE_M * Q_TILES;  // query rows per work unit
 constexpr int MAX_Q_GROUPS = 512;  // per (batch, head); bounds the per-CTA prefix table
 constexpr int MAX_GRID = 256;      // CTAs of one attention launch (the schedule is a kernel parameter)
 
+// Status-word bit of the bounds-checked build: an index check failed (the access
+// was skipped).  Bit 0 is a device wait that ran out (dz_ptx.cuh).
+constexpr int DZ_DEV_BOUNDS = 2;
+
+// Index check of the bounds-checked build (DZ_DEBUG_BOUNDS): whether element i of a
+// buffer of n elements may be accessed.  A failed check records DZ_DEV_BOUNDS in the
+// status word and the caller skips the access.  Other builds compile it away.
+__device__ __forceinline__ bool in_bounds(long long i, long long n, int* status) {
+#ifdef DZ_DEBUG_BOUNDS
+  if (i >= 0 && i < n) return true;
+  atomicOr(status, DZ_DEV_BOUNDS);
+  return false;
+#else
+  (void)i;
+  (void)n;
+  (void)status;
+  return true;
+#endif
+}
+
 // Rotary tables: (cos, sin) as float2 for every (axis position, pair of that axis).
 struct RopeTables {
   const float2* tab;
   int off_t, off_h, off_w;  // element offsets of the t, h and w tables
   int pt, ph, pw;           // pairs per axis
+  int n;                    // entries of tab
 };
 
 // Token-to-position rule of a run of whole chunks (see dz.h): token s of the
@@ -53,6 +74,14 @@ __device__ __forceinline__ int rope_index(const RopeTables& r, int j, int t, int
   const int pth = r.pt + r.ph;
   return j < r.pt ? r.off_t + t * r.pt + j
                   : (j < pth ? r.off_h + h * r.ph + (j - r.pt) : r.off_w + w * r.pw + (j - pth));
+}
+
+// rope_index checked against the table in the bounds-checked build (entry 0 when
+// the check fails).
+__device__ __forceinline__ int rope_index_checked(const RopeTables& r, int j, int t, int h, int w,
+                                                  int* status) {
+  const int i = rope_index(r, j, t, h, w);
+  return in_bounds(i, r.n, status) ? i : 0;
 }
 
 // One rotated pair (two bf16 in a 32-bit word) in fp32, rounded to bf16.  Used
@@ -147,16 +176,17 @@ __host__ __device__ __forceinline__ int unit_tile_count(const SchedGeom& g, int 
 // Kernel launchers (defined in the .cu files; return cudaGetLastError()).
 // ---------------------------------------------------------------------------
 cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int B, int rows,
-                           int H, int cap, int dst_row0, cudaStream_t stream);
+                           int H, int cap, int dst_row0, int* status, cudaStream_t stream);
 #ifdef DZ_TEST_HOOKS
 // Test builds only: x[0:n] = value.
 cudaError_t launch_fill_i32(int* x, size_t n, int value, cudaStream_t stream);
 #endif
 
 // Rotates x into y (and x1 into y1 when x1 is not null) for B x S tokens; with
-// period > 0 token s is rotated at the position of token s % period.
+// period > 0 token s is rotated at the position of token s % period.  `status`
+// receives the bounds-checked build's index faults.
 cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const ChunkGeom& g,
-                          int first_chunk, const RopeTables& r, cudaStream_t stream,
+                          int first_chunk, const RopeTables& r, int* status, cudaStream_t stream,
                           const void* x1 = nullptr, void* y1 = nullptr, int period = 0);
 
 struct AttnLaunch {
@@ -166,6 +196,11 @@ struct AttnLaunch {
   float* ws;
   int* counters;
   int* status;
+  // extents for the bounds-checked build: out elements (B * Sq * H * 128; lse has
+  // a 128th of that), partial-result slots of ws, split counters
+  long long out_elems;
+  int ws_slots;
+  long long n_counters;
   RopeTables rope;
   ChunkGeom geom;
   SchedGeom sched;

@@ -16,13 +16,20 @@ __global__ void __launch_bounds__(256) kv_copy_kernel(const uint4* __restrict__ 
                                                       uint4* __restrict__ ck,
                                                       uint4* __restrict__ cv, int B,
                                                       long long span_vecs, long long src_stride,
-                                                      long long dst_stride, long long dst_off) {
+                                                      long long dst_stride, long long dst_off,
+                                                      int* status) {
   const int which = blockIdx.y / B;  // 0 = keys, 1 = values
   const int b = blockIdx.y - which * B;
   const uint4* src = (which == 0 ? k : v) + static_cast<long long>(b) * src_stride;
   uint4* dst = (which == 0 ? ck : cv) + static_cast<long long>(b) * dst_stride + dst_off;
   const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
   long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+#ifdef DZ_DEBUG_BOUNDS
+  // the destination rows must lie inside this batch item's cache rows
+  if (!in_bounds(dst_off + span_vecs - 1, dst_stride, status)) return;
+#else
+  (void)status;
+#endif
   for (; i + 3 * step < span_vecs; i += 4 * step) {
     const uint4 a0 = src[i], a1 = src[i + step], a2 = src[i + 2 * step], a3 = src[i + 3 * step];
     dst[i] = a0;
@@ -34,7 +41,7 @@ __global__ void __launch_bounds__(256) kv_copy_kernel(const uint4* __restrict__ 
 }
 
 cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int B, int rows,
-                           int H, int cap, int dst_row0, cudaStream_t stream) {
+                           int H, int cap, int dst_row0, int* status, cudaStream_t stream) {
   const long long row_vecs = static_cast<long long>(H) * HEAD_DIM * 2 / 16;
   const long long span = row_vecs * rows;
   int dev = 0, sms = 148;
@@ -48,7 +55,7 @@ cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int
   dim3 grid(gx, 2 * B);
   kv_copy_kernel<<<grid, 256, 0, stream>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(ck),
-      static_cast<uint4*>(cv), B, span, span, row_vecs * cap, row_vecs * dst_row0);
+      static_cast<uint4*>(cv), B, span, span, row_vecs * cap, row_vecs * dst_row0, status);
   return cudaGetLastError();
 }
 
@@ -70,7 +77,8 @@ constexpr int ROPE_UNROLL = 8;  // chunks per thread per pass: 64 heads with 128
 __global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, uint4* y0,
                                                             const uint4* x1, uint4* y1, int S,
                                                             int H, ChunkGeom g, int first_chunk,
-                                                            int period, RopeTables r) {
+                                                            int period, RopeTables r,
+                                                            int* status) {
   const long long token = blockIdx.x;  // b * S + s
   int s = static_cast<int>(token % S);
   if (period > 0) s %= period;
@@ -82,7 +90,7 @@ __global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, uin
   const int j0 = (threadIdx.x & 15) * 4;  // ROPE_BLOCK is a multiple of 16
   float2 cs[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) cs[k] = __ldg(r.tab + rope_index(r, j0 + k, t, hh, w));
+  for (int k = 0; k < 4; ++k) cs[k] = __ldg(r.tab + rope_index_checked(r, j0 + k, t, hh, w, status));
   for (int i0 = threadIdx.x; i0 < nvec; i0 += ROPE_BLOCK * ROPE_UNROLL) {
     uint4 v[ROPE_UNROLL];
 #pragma unroll
@@ -101,14 +109,14 @@ __global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, uin
 }
 
 cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const ChunkGeom& g,
-                          int first_chunk, const RopeTables& r, cudaStream_t stream,
+                          int first_chunk, const RopeTables& r, int* status, cudaStream_t stream,
                           const void* x1, void* y1, int period) {
   const long long tokens = static_cast<long long>(B) * S;
   if (tokens <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(tokens), x1 ? 2 : 1);
   rope3d_kernel<<<grid, ROPE_BLOCK, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
                                           static_cast<const uint4*>(x1), static_cast<uint4*>(y1),
-                                          S, H, g, first_chunk, period, r);
+                                          S, H, g, first_chunk, period, r, status);
   return cudaGetLastError();
 }
 

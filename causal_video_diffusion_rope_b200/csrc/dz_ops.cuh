@@ -10,7 +10,7 @@ struct QkvLaunch {
   CUtensorMap tm_x, tm_w;  // x [M][K], w [3*H*128][K], bf16, 64 x 256 / 64 x bn boxes, SW128
   void *q, *k, *v;         // [M][H][128]
   void *ck, *cv;           // cache or null
-  int cache_cap, cache_row0;
+  int cache_cap, cache_row0, cache_batch;
   int M, S, H, K;
   int bn;  // output features per tile (qkv_tile_n)
   RopeTables rope;

@@ -59,6 +59,7 @@ struct __align__(64) QkvParams {
   __nv_bfloat16 *ck, *cv;  // cache (null: no append)
   int cache_cap, cache_row0;
   int M, S, H, K, N;
+  int cache_batch;  // batch items of the cache (bounds-checked build)
   int bn;  // features per tile
   int m_tiles, n_tiles;
   RopeTables rope;
@@ -198,13 +199,18 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
       const float2* gt = p.rope.tab + p.rope.off_t + p.stage_t0 * p.rope.pt;
       const float2* gh = p.rope.tab + p.rope.off_h;
       const float2* gw = p.rope.tab + p.rope.off_w;
-      for (int i = tid - 64; i < nt_ + nh + nw; i += QTHREADS - 64)
-        st_tab[i] = i < nt_ ? gt[i] : (i < nt_ + nh ? gh[i - nt_] : gw[i - nt_ - nh]);
+      for (int i = tid - 64; i < nt_ + nh + nw; i += QTHREADS - 64) {
+        const long long gi = i < nt_ ? p.rope.off_t + static_cast<long long>(p.stage_t0) * p.rope.pt + i
+                                     : (i < nt_ + nh ? p.rope.off_h + i - nt_ : p.rope.off_w + i - nt_ - nh);
+        if (in_bounds(gi, p.rope.n, p.status))
+          st_tab[i] = i < nt_ ? gt[i] : (i < nt_ + nh ? gh[i - nt_] : gw[i - nt_ - nh]);
+      }
       named_bar_sync(1, QTHREADS - 64);
       rope.tab = st_tab;
       rope.off_t = -p.stage_t0 * p.rope.pt;
       rope.off_h = nt_;
       rope.off_w = nt_ + nh;
+      rope.n = nt_ + nh + nw;
     }
     int lt = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++lt) {
@@ -234,7 +240,8 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
         float2 cs[8];
         if (sec < 2) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) cs[i] = rope.tab[rope_index(rope, d0 / 2 + i, t, hh, w)];
+          for (int i = 0; i < 8; ++i)
+            cs[i] = rope.tab[rope_index_checked(rope, d0 / 2 + i, t, hh, w, p.status)];
         }
         uint32_t pk[8];
         if (sec < 2) {
@@ -251,14 +258,16 @@ __global__ void __launch_bounds__(QTHREADS, 1) qkv_rope_kernel(const __grid_cons
             pk[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
         }
         if (valid) {
-          __nv_bfloat16* dst = (sec == 0 ? p.q : (sec == 1 ? p.k : p.v)) +
-                               (static_cast<size_t>(m) * p.H + head) * HEAD_DIM + d0;
-          store_piece(dst, pk);
+          const long long oi = (static_cast<long long>(m) * p.H + head) * HEAD_DIM + d0;
+          if (in_bounds(oi + 15, static_cast<long long>(p.M) * p.H * HEAD_DIM, p.status))
+            store_piece((sec == 0 ? p.q : (sec == 1 ? p.k : p.v)) + oi, pk);
           if (sec > 0 && p.ck) {
-            __nv_bfloat16* cdst = (sec == 1 ? p.ck : p.cv) +
-                                  ((static_cast<size_t>(bb) * p.cache_cap + p.cache_row0 + s) * p.H +
-                                   head) * HEAD_DIM + d0;
-            store_piece(cdst, pk);
+            const long long ci =
+                ((static_cast<long long>(bb) * p.cache_cap + p.cache_row0 + s) * p.H + head) * HEAD_DIM + d0;
+            if (in_bounds(ci + 15,
+                          static_cast<long long>(p.cache_batch) * p.cache_cap * p.H * HEAD_DIM,
+                          p.status))
+              store_piece((sec == 1 ? p.ck : p.cv) + ci, pk);
           }
         }
         tmem_wait_ld();
@@ -318,6 +327,7 @@ cudaError_t launch_qkv_rope(const QkvLaunch& a, cudaStream_t stream) {
   p.cv = static_cast<__nv_bfloat16*>(a.cv);
   p.cache_cap = a.cache_cap;
   p.cache_row0 = a.cache_row0;
+  p.cache_batch = a.cache_batch;
   p.M = a.M;
   p.S = a.S;
   p.H = a.H;

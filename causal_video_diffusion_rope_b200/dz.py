@@ -23,6 +23,7 @@ DZ_ERR_CAPACITY = 4
 DZ_ERR_CUDA = 5
 DZ_ERR_UNSUPPORTED = 6
 DZ_ERR_TIMEOUT = 7
+DZ_ERR_BOUNDS = 8
 
 DZ_MODE_DECODE = 0
 DZ_MODE_TEACHER_FORCING = 1

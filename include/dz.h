@@ -53,7 +53,8 @@ typedef enum {
   DZ_ERR_CAPACITY = 4,    /* cache or handle capacity would be exceeded        */
   DZ_ERR_CUDA = 5,        /* a CUDA runtime/driver call failed                 */
   DZ_ERR_UNSUPPORTED = 6, /* valid request this build does not implement       */
-  DZ_ERR_TIMEOUT = 7      /* a device-side bounded wait ran out                */
+  DZ_ERR_TIMEOUT = 7,     /* a device-side bounded wait ran out                */
+  DZ_ERR_BOUNDS = 8       /* a device index check failed (bounds-checked build) */
 } dz_status;
 
 typedef struct dz_attn* dz_attn_t; /* opaque handle */
@@ -298,8 +299,10 @@ dz_status dz_chunk_attn_forward_noalloc(const dz_attn_desc* desc, const void* q,
 
 /* Synchronise `stream`, read and clear the handle's device status word.
  * Returns DZ_ERR_TIMEOUT if a kernel's bounded wait ran out since the last
- * read (that call's output is incomplete), DZ_ERR_CUDA on a CUDA error, else
- * DZ_OK.  With a NULL handle it reads and clears the status word of the
+ * read (that call's output is incomplete), DZ_ERR_BOUNDS if a kernel of the
+ * bounds-checked test build found an index outside its buffer (the access was
+ * skipped; never returned by the product build), DZ_ERR_CUDA on a CUDA error,
+ * else DZ_OK.  With a NULL handle it reads and clears the status word of the
  * allocation-free calls (dz_chunk_attn_forward_noalloc) on the current device
  * instead (DZ_OK if none was made there). */
 dz_status dz_attn_sync_status(dz_attn_t handle, void* stream);
