@@ -10,18 +10,19 @@
 //   dq = R^T dqr,  dk = R^T dkr.
 // Two kernels recompute S and dP instead of exchanging partial sums:
 //   bwd_dq_kernel   one CTA per (batch, head, 128-query tile): over the key tiles
-//                   it sees, S = Q K^T and dP = dO V^T (both operands K-major in
-//                   shared memory), dS in registers, written as bf16 over S in
-//                   TMEM, then dQ += dS K with dS read from TMEM;
+//                   it sees, S = Q K^T and dP = dO V^T on whole 128-key tiles (both
+//                   operands K-major in shared memory), dS in registers, written as
+//                   bf16 into one of two TMEM buffers, then dQ += dS K with dS read
+//                   from TMEM; the next tile's S and dP run while dS is computed;
 //   bwd_dkv_kernel  one CTA per (batch, head, 128-key tile): over the query tiles
 //                   that see it, S^T = K Q^T and dP^T = V dO^T, P^T and dS^T
 //                   written as bf16 over them in TMEM, then dV += P^T dO and
 //                   dK += dS^T Q.
-// Each has a TMA warp (2-stage ring of the streamed tiles), an MMA warp and eight
-// compute warps: two per TMEM lane quarter, one thread per tile row, each of the
-// two taking 32 of a half-tile's 64 columns.  A streamed tile is taken in two
-// halves of 64 rows with two TMEM buffers, so that the products of one half run
-// while the compute warps turn the other half's scores into bf16 operands.  Each
+// Each has a TMA warp, an MMA warp and eight compute warps: two per TMEM lane
+// quarter, one thread per tile row.  In bwd_dkv_kernel a streamed tile is taken in
+// two halves of 64 rows with two TMEM buffers (2-stage ring), so that the products
+// of one half run while the compute warps turn the other half's scores into bf16
+// operands; each of a lane quarter's two warps takes 32 of a half's 64 columns.  Each
 // thread writes its bf16 operands over its own fp32 columns, so a half's operand
 // occupies columns [0, 16) and [32, 48) of its region (see mma_tmem_a64).  The rotation back (R^T) and the 1/sqrt(128) are applied to the fp32
 // accumulators in the epilogue.
@@ -175,16 +176,46 @@ constexpr uint32_t HALF_ROWS_OFF = (64 * 128) >> 4;  // 64 rows of 128 bytes, in
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// dQ: one CTA per (batch, head, query tile).  TMEM: S [0,128) (dS bf16 over its
-// first 64 columns), dP [128,256), dQ [256,384).
+// dQ: one CTA per (batch, head, query tile), whole 128-key tiles.  TMEM: S
+// [0,128), dP [128,256), dQ [256,384), dS (bf16) in two buffers [384,448) and
+// [448,512).  Shared memory: Q and dO resident, K tiles in a 3-stage ring (a K
+// tile is read by S and, a tile later, by dQ), V tiles in a 2-stage ring (read by
+// dP only).  Per key tile t the MMA warp issues S(t) and dP(t) as soon as the
+// compute warps hold S(t-1) and dP(t-1) in registers, then dQ += dS(t-1) K(t-1)
+// once they have written dS(t-1); so the products of tile t run while the compute
+// warps turn tile t-1's scores into dS.
 // ---------------------------------------------------------------------------
+constexpr int DQ_KSTAGES = 3, DQ_VSTAGES = 2;
+constexpr int DQ_SM_Q = 0, DQ_SM_DO = BTILE;
+constexpr int DQ_SM_K = 2 * BTILE;
+constexpr int DQ_SM_V = DQ_SM_K + DQ_KSTAGES * BTILE;
+constexpr int DQ_SM_BAR = DQ_SM_V + DQ_VSTAGES * BTILE;
+constexpr int DQ_SM_MISC = DQ_SM_BAR + 256;
+constexpr int DQ_SMEM_BYTES = DQ_SM_MISC + 64 + 1024;
+static_assert(DQ_SMEM_BYTES <= 232448, "shared memory");
+enum {
+  DQ_FIX = 0,                            // Q and dO landed
+  DQ_KFULL = 1,                          // [3] K stage landed
+  DQ_KEMPTY = DQ_KFULL + DQ_KSTAGES,     // [3] K stage read by S and dQ
+  DQ_VFULL = DQ_KEMPTY + DQ_KSTAGES,     // [2] V stage landed
+  DQ_VEMPTY = DQ_VFULL + DQ_VSTAGES,     // [2] V stage read by dP
+  DQ_SDP = DQ_VEMPTY + DQ_VSTAGES,       // S and dP of the tile in TMEM
+  DQ_READ = DQ_SDP + 1,                  // compute warps hold S, dP in registers (256)
+  DQ_DS = DQ_READ + 1,                   // [2] dS written into buffer u (256)
+  DQ_DSFREE = DQ_DS + 2,                 // [2] dQ product done reading buffer u
+  DQ_ACC = DQ_DSFREE + 2,
+  DQ_DRAIN = DQ_ACC + 1,
+  DQ_COUNT = DQ_DRAIN + 1
+};
+static_assert(DQ_COUNT * 8 <= 256, "barrier area");
+
 __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_constant__ BwdParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + BSM_BAR);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + BSM_MISC);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + BSM_MISC + 4);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + DQ_SM_BAR);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + DQ_SM_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + DQ_SM_MISC + 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = blockIdx.x % p.n_tiles;
   const int bh = blockIdx.x / p.n_tiles;
@@ -192,17 +223,23 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
   const int q0 = qt * BT;
 
   if (tid == 0) {
-    mbar_init(&bar[BB_FIX], 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar[BB_FULL + s], 1);
-      mbar_init(&bar[BB_EMPTY + s], 1);
+    mbar_init(&bar[DQ_FIX], 1);
+    for (int s = 0; s < DQ_KSTAGES; ++s) {
+      mbar_init(&bar[DQ_KFULL + s], 1);
+      mbar_init(&bar[DQ_KEMPTY + s], 1);
     }
+    for (int s = 0; s < DQ_VSTAGES; ++s) {
+      mbar_init(&bar[DQ_VFULL + s], 1);
+      mbar_init(&bar[DQ_VEMPTY + s], 1);
+    }
+    mbar_init(&bar[DQ_SDP], 1);
+    mbar_init(&bar[DQ_READ], BCOMPUTE);
     for (int u = 0; u < 2; ++u) {
-      mbar_init(&bar[BB_SDP + u], 1);
-      mbar_init(&bar[BB_READY + u], BCOMPUTE);
+      mbar_init(&bar[DQ_DS + u], BCOMPUTE);
+      mbar_init(&bar[DQ_DSFREE + u], 1);
     }
-    mbar_init(&bar[BB_ACC], 1);
-    mbar_init(&bar[BB_DRAIN], 1);
+    mbar_init(&bar[DQ_ACC], 1);
+    mbar_init(&bar[DQ_DRAIN], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -217,73 +254,81 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_expect_tx(&bar[BB_FIX], 2 * BTILE);
-      tile_load(smem + BSM_FIXED0, &p.tm_q, &bar[BB_FIX], h, q0, b);
-      tile_load(smem + BSM_FIXED1, &p.tm_do, &bar[BB_FIX], h, q0, b);
-      uint32_t it = 0;
+      mbar_expect_tx(&bar[DQ_FIX], 2 * BTILE);
+      tile_load(smem + DQ_SM_Q, &p.tm_q, &bar[DQ_FIX], h, q0, b);
+      tile_load(smem + DQ_SM_DO, &p.tm_do, &bar[DQ_FIX], h, q0, b);
+      uint32_t nk = 0, nv = 0;  // K and V tiles issued
       for (int kt = 0; kt < p.n_tiles; ++kt) {
         if (!pair_visible(p, qt, kt)) continue;
-        const int st = it & 1;
-        if (!mbar_wait(&bar[BB_EMPTY + st], ((it >> 1) & 1) ^ 1, abort_flag, p.status)) break;
-        uint8_t* ring = smem + BSM_RING + st * 2 * BTILE;
-        mbar_expect_tx(&bar[BB_FULL + st], 2 * BTILE);
-        tile_load(ring, &p.tm_k, &bar[BB_FULL + st], h, kt * BT, b);
-        tile_load(ring + BTILE, &p.tm_v, &bar[BB_FULL + st], h, kt * BT, b);
-        ++it;
+        const int ks = nk % DQ_KSTAGES, vs = nv % DQ_VSTAGES;
+        if (!mbar_wait(&bar[DQ_KEMPTY + ks], ((nk / DQ_KSTAGES) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_expect_tx(&bar[DQ_KFULL + ks], BTILE);
+        tile_load(smem + DQ_SM_K + ks * BTILE, &p.tm_k, &bar[DQ_KFULL + ks], h, kt * BT, b);
+        ++nk;
+        if (!mbar_wait(&bar[DQ_VEMPTY + vs], ((nv / DQ_VSTAGES) & 1) ^ 1, abort_flag, p.status)) break;
+        mbar_expect_tx(&bar[DQ_VFULL + vs], BTILE);
+        tile_load(smem + DQ_SM_V + vs * BTILE, &p.tm_v, &bar[DQ_VFULL + vs], h, kt * BT, b);
+        ++nv;
       }
-      mbar_drain(&bar[BB_FIX], 0);
-      for (uint32_t j = (it > 2 ? it - 2 : 0); j < it; ++j) mbar_drain(&bar[BB_FULL + (j & 1)], (j >> 1) & 1);
+      // every issued copy has landed before the CTA exits
+      mbar_drain(&bar[DQ_FIX], 0);
+      for (uint32_t j = (nk > DQ_KSTAGES ? nk - DQ_KSTAGES : 0); j < nk; ++j)
+        mbar_drain(&bar[DQ_KFULL + j % DQ_KSTAGES], (j / DQ_KSTAGES) & 1);
+      for (uint32_t j = (nv > DQ_VSTAGES ? nv - DQ_VSTAGES : 0); j < nv; ++j)
+        mbar_drain(&bar[DQ_VFULL + j % DQ_VSTAGES], (j / DQ_VSTAGES) & 1);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t id_n64 = idesc_bf16(BT, 64, false);
+      const uint32_t id_qk = idesc_bf16(BT, BT, false);
       const uint32_t id_mn = idesc_bf16(BT, HEAD_DIM, true);
-      const uint32_t q_lo = desc_lo(smem_u32(smem + BSM_FIXED0), 16);
-      const uint32_t do_lo = desc_lo(smem_u32(smem + BSM_FIXED1), 16);
-      bool ok = mbar_wait(&bar[BB_FIX], 0, abort_flag, p.status);
+      const uint32_t q_lo = desc_lo(smem_u32(smem + DQ_SM_Q), 16);
+      const uint32_t do_lo = desc_lo(smem_u32(smem + DQ_SM_DO), 16);
+      bool ok = mbar_wait(&bar[DQ_FIX], 0, abort_flag, p.status);
       tc_fence_after();
-      // half-step j = 2 * (key tile ordinal) + half; TMEM buffer = half
-      auto issue_dq = [&](uint32_t jj) {  // dQ += dS K over the 64 keys of half-step jj
-        const int hf = jj & 1, st = (jj >> 1) & 1;
-        const uint32_t k_mn = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), BHALF);
-        mma_tmem_a64(tmem + 256, tmem + 128 * hf, k_mn + hf * HALF_ROWS_OFF, id_mn, jj > 0);
-        if (hf == 1) mma_commit(&bar[BB_EMPTY + st]);
+      // dQ += dS(t) K(t): A = dS (bf16 pairs in TMEM), B = K tile MN-major (dims
+      // contiguous; the two 64-dim halves LBO apart)
+      auto issue_dq = [&](uint32_t tt) -> bool {
+        const int u = tt & 1, ks = tt % DQ_KSTAGES;
+        if (!mbar_wait(&bar[DQ_DS + u], (tt >> 1) & 1, abort_flag, p.status)) return false;
+        tc_fence_after();
+        const uint32_t k_mn = desc_lo(smem_u32(smem + DQ_SM_K + ks * BTILE), BHALF);
+#pragma unroll
+        for (int kk = 0; kk < BT / 16; ++kk)
+          mma_ts(tmem + 256, tmem + 384 + 64 * u + kk * 8, desc_join(k_mn + ((kk * 16 * 128) >> 4)),
+                 id_mn, (tt > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bar[DQ_DSFREE + u]);
+        mma_commit(&bar[DQ_KEMPTY + ks]);
+        return true;
       };
       uint32_t t = 0;  // visible key tiles so far
       for (int kt = 0; ok && kt < p.n_tiles; ++kt) {
         if (!pair_visible(p, qt, kt)) continue;
-        const int st = t & 1;
-        const uint32_t k_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE), 16);
-        const uint32_t v_lo = desc_lo(smem_u32(smem + BSM_RING + st * 2 * BTILE + BTILE), 16);
-        for (int hf = 0; hf < 2; ++hf) {
-          const uint32_t jj = 2 * t + hf;
-          if (jj >= 2) {  // buffer hf is free once half-step jj - 2 is turned into dS
-            if (!mbar_wait(&bar[BB_READY + hf], ((jj - 2) >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-            issue_dq(jj - 2);
-          }
-          if (hf == 0) {  // the key tile (waited after the previous tile's dQ went out)
-            if (!mbar_wait(&bar[BB_FULL + st], (t >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-            tc_fence_after();
-          }
-          mma_kmajor(tmem + 128 * hf, q_lo, k_lo + hf * HALF_ROWS_OFF, id_n64);        // S
-          mma_kmajor(tmem + 128 * hf + 64, do_lo, v_lo + hf * HALF_ROWS_OFF, id_n64);  // dP
-          mma_commit(&bar[BB_SDP + hf]);
+        const int ks = t % DQ_KSTAGES, vs = t % DQ_VSTAGES;
+        if (!mbar_wait(&bar[DQ_KFULL + ks], (t / DQ_KSTAGES) & 1, abort_flag, p.status) ||
+            !mbar_wait(&bar[DQ_VFULL + vs], (t / DQ_VSTAGES) & 1, abort_flag, p.status) ||
+            (t > 0 && !mbar_wait(&bar[DQ_READ], (t - 1) & 1, abort_flag, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        mma_kmajor(tmem, q_lo, desc_lo(smem_u32(smem + DQ_SM_K + ks * BTILE), 16), id_qk);          // S
+        mma_kmajor(tmem + 128, do_lo, desc_lo(smem_u32(smem + DQ_SM_V + vs * BTILE), 16), id_qk);  // dP
+        mma_commit(&bar[DQ_SDP]);
+        mma_commit(&bar[DQ_VEMPTY + vs]);
+        if (t > 0 && !issue_dq(t - 1)) {
+          ok = false;
+          break;
         }
         ++t;
       }
-      for (uint32_t jj = (2 * t >= 2 ? 2 * t - 2 : 0); ok && jj < 2 * t; ++jj) {
-        if (!mbar_wait(&bar[BB_READY + (jj & 1)], (jj >> 1) & 1, abort_flag, p.status)) break;
-        tc_fence_after();
-        issue_dq(jj);
-      }
-      mma_commit(&bar[BB_ACC]);
-      mma_commit(&bar[BB_DRAIN]);
-      mbar_drain(&bar[BB_DRAIN], 0);
+      if (ok && t > 0) ok = issue_dq(t - 1);
+      mma_commit(&bar[DQ_ACC]);
+      mma_commit(&bar[DQ_DRAIN]);
+      mbar_drain(&bar[DQ_DRAIN], 0);
     }
   } else {
     const int quarter = warp & 3;
-    const int cg = (warp - 2) >> 2;  // column group: columns [32 cg, 32 cg + 32) of a half
+    const int cg = (warp - 2) >> 2;  // column group: key columns [64 cg, 64 cg + 64) of a tile
     const int r = 32 * quarter + lane;
     const uint32_t la = static_cast<uint32_t>(32 * quarter) << 16;
     const int s = q0 + r;
@@ -300,38 +345,54 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
     bool ok = true;
     for (int kt = 0; ok && kt < p.n_tiles; ++kt) {
       if (!pair_visible(p, qt, kt)) continue;
-      const int k0 = kt * BT;
-      for (int hf = 0; hf < 2; ++hf) {
-        const uint32_t hs = 2 * it + hf;  // half-step
-        if (!mbar_wait(&bar[BB_SDP + hf], (hs >> 1) & 1, abort_flag, p.status)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t col = 128 * hf + 32 * cg;
-        uint32_t sv[32], dp[32];
-        tmem_ld32(tmem + la + col, sv);
-        tmem_ld32(tmem + la + col + 64, dp);
-        tmem_wait_ld();
-        const int col0 = k0 + 64 * hf + 32 * cg;
-        const uint32_t keep = range_bits(a0 - col0, a1 - col0) | range_bits(b0 - col0, b1 - col0);
-        uint32_t pk[16];
+      if (!mbar_wait(&bar[DQ_SDP], it & 1, abort_flag, p.status)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[64], dp[64];
+      {
+        uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv);
+        uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(sv + 32);
+        uint32_t (&d0)[32] = *reinterpret_cast<uint32_t(*)[32]>(dp);
+        uint32_t (&d1)[32] = *reinterpret_cast<uint32_t(*)[32]>(dp + 32);
+        tmem_ld32(tmem + la + 64 * cg, s0);
+        tmem_ld32(tmem + la + 64 * cg + 32, s1);
+        tmem_ld32(tmem + la + 128 + 64 * cg, d0);
+        tmem_ld32(tmem + la + 128 + 64 * cg + 32, d1);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bar[DQ_READ]);  // S and dP of this tile may now be overwritten
+      const int col0 = kt * BT + 64 * cg;
+      uint32_t pk[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int c0 = col0 + 32 * hh;
+        const uint32_t keep = range_bits(a0 - c0, a1 - c0) | range_bits(b0 - c0, b1 - c0);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           float d2[2];
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int j = 2 * i + e;
-            const float pe = ex2(__uint_as_float(sv[j]) * p.scale_log2 - lse2);
-            d2[e] = ((keep >> j) & 1u) ? pe * (__uint_as_float(dp[j]) - dsum) : 0.f;
+            const float pe = ex2(__uint_as_float(sv[32 * hh + j]) * p.scale_log2 - lse2);
+            d2[e] = ((keep >> j) & 1u) ? pe * (__uint_as_float(dp[32 * hh + j]) - dsum) : 0.f;
           }
-          pk[i] = pack_bf16x2(d2[0], d2[1]);
+          pk[16 * hh + i] = pack_bf16x2(d2[0], d2[1]);
         }
-        tmem_st16(tmem + la + col, pk);  // dS over this thread's own S columns
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bar[BB_READY + hf]);
       }
+      const int u = it & 1;
+      // buffer u is free once the dQ product of tile it - 2 has read it
+      if (it >= 2 && !mbar_wait(&bar[DQ_DSFREE + u], ((it - 2) >> 1) & 1, abort_flag, p.status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st32(tmem + la + 384 + 64 * u + 32 * cg, pk);  // dS, keys [64 cg, 64 cg + 64)
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bar[DQ_DS + u]);
       ++it;
     }
-    if (ok && mbar_wait(&bar[BB_ACC], 0, abort_flag, p.status)) {
+    if (ok && mbar_wait(&bar[DQ_ACC], 0, abort_flag, p.status)) {
       tc_fence_after();
       int t, hh, w;
       bpos(p, s_eff, t, hh, w);
@@ -617,7 +678,7 @@ cudaError_t launch_backward(const BwdLaunch& a, cudaStream_t stream) {
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
     cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         BSMEM_BYTES);
+                                         DQ_SMEM_BYTES);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                BSMEM_BYTES);
@@ -651,7 +712,7 @@ cudaError_t launch_backward(const BwdLaunch& a, cudaStream_t stream) {
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));
   p.status = a.status;
   const unsigned grid = static_cast<unsigned>(a.B * a.H * p.n_tiles);
-  bwd_dq_kernel<<<grid, BTHREADS, BSMEM_BYTES, stream>>>(p);
+  bwd_dq_kernel<<<grid, BTHREADS, DQ_SMEM_BYTES, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   bwd_dkv_kernel<<<grid, BTHREADS, BSMEM_BYTES, stream>>>(p);
