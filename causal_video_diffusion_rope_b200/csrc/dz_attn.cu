@@ -9,7 +9,9 @@
 // Design (one persistent CTA per SM, 384 threads = 12 warps, 1 CTA/SM; 12 warps
 // keep 3 warps per SM sub-partition, which leaves up to 168 registers a thread):
 //   warp 0        TMA producer: Q tiles of the current unit, then K and V tiles
-//                 through a 2-stage ring (128B-swizzled, K-major rows of 128 dims).
+//                 through a 2-stage ring (128B-swizzled, K-major rows of 128 dims);
+//                 one commit after each tile's QK products frees its K stage and the
+//                 previous tile's V stage (those PV products precede it in the queue).
 //   warp 1        TMEM owner (512 columns) and single-thread tcgen05.mma issuer.
 //   warps 2-3     rotary gate: rotates the Q tiles and the call's own K tiles in
 //                 shared memory (RoPE fused into the tile load, two rows per
@@ -81,10 +83,9 @@ enum {
   B_K_FULL = 3,                     // K tile landed (tiles used as loaded)
   B_K_RAW = B_K_FULL + KV_STAGES,   // K tile landed (tiles the rotary gate must rotate)
   B_K_READY = B_K_RAW + KV_STAGES,  // rotated K tile released to the tensor core
-  B_K_EMPTY = B_K_READY + KV_STAGES,
+  B_K_EMPTY = B_K_READY + KV_STAGES,  // tile's QK products done (and the previous tile's PV)
   B_V_FULL = B_K_EMPTY + KV_STAGES,
-  B_V_EMPTY = B_V_FULL + KV_STAGES,
-  B_S_FULL = B_V_EMPTY + KV_STAGES,
+  B_S_FULL = B_V_FULL + KV_STAGES,
   B_P_FULL = B_S_FULL + Q_TILES,
   B_O_FULL = B_P_FULL + Q_TILES,
   B_O_FREE = B_O_FULL + Q_TILES,
@@ -432,7 +433,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bar[B_K_READY + s], ROPE_THREADS);
       mbar_init(&bar[B_K_EMPTY + s], 1);
       mbar_init(&bar[B_V_FULL + s], 1);
-      mbar_init(&bar[B_V_EMPTY + s], 1);
     }
     for (int q = 0; q < Q_TILES; ++q) {
       mbar_init(&bar[B_S_FULL + q], 1);
@@ -548,7 +548,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tma_load_4d(sK + st * TILE_BYTES + HALF_BYTES, mk, kb, 64, h, kt.row0, b);
           if (kt.rope) ++kr_cnt[st]; else ++kf_cnt[st];
           ++k_iss;
-          if (!mbar_wait(&bar[B_V_EMPTY + st], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+          // the V stage held V(t - 2), whose products were issued before QK(t - 1): the
+          // single commit after tile t - 1's QK products covers them
+          if (v_iss >= 2) {
+            const uint32_t tp = v_iss - 1;
+            if (!mbar_wait(&bar[B_K_EMPTY + tp % KV_STAGES], (tp / KV_STAGES) & 1, abort_flag, p.status)) {
+              ok = false;
+              break;
+            }
+          }
           mbar_expect_tx(&bar[B_V_FULL + st], TILE_BYTES);
           tma_load_4d(sV + st * TILE_BYTES, mv, &bar[B_V_FULL + st], 0, h, kt.row0, b);
           tma_load_4d(sV + st * TILE_BYTES + HALF_BYTES, mv, &bar[B_V_FULL + st], 64, h, kt.row0, b);
@@ -638,7 +646,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
               }
               tc_fence_after();
               issue_pv(q, pst, i > 1);
-              if (q == Q_TILES - 1) mma_commit(&bar[B_V_EMPTY + pst]);
               issue_qk(q, st);
               mma_commit(&bar[B_S_FULL + q]);
             }
@@ -667,7 +674,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_commit(&bar[B_O_FULL + q]);
         }
         if (!ok) break;
-        mma_commit(&bar[B_V_EMPTY + pst]);
         ++seg_i;
       }
       // every issued MMA has completed before TMEM is released
