@@ -209,6 +209,55 @@ def make_inputs(w: Workload, seed: int, cache_capacity: Optional[int] = None) ->
     return out
 
 
+# Multipliers of the E4M3 operands (one per tensor, powers of two): |q| stays
+# below ~6 and |k| below ~18 on the K x 3 heads, so the codes stay under 448.
+E4M3_Q_SCALE = 64.0
+E4M3_K_SCALE = 16.0
+
+
+def normal_e4m3(rng: np.random.Generator, shape, multiplier: float,
+                scale: Optional[np.ndarray] = None) -> np.ndarray:
+    """Standard normals drawn in float32 (optionally scaled per head), times
+    ``multiplier``, cast to float8_e4m3fn by torch (nearest, ties to even);
+    returns the uint8 codes.  Values are clipped to +-440 first (the cast gives
+    NaN past the format's range)."""
+    import torch
+
+    x = rng.standard_normal(size=shape, dtype=np.float32)
+    if scale is not None:
+        x = x * scale.astype(np.float32)[None, None, :, None]
+    x = np.clip(x * np.float32(multiplier), -440.0, 440.0).astype(np.float32)
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def make_inputs_e4m3(w: Workload, seed: int,
+                     cache_capacity: Optional[int] = None) -> Dict[str, np.ndarray]:
+    """Inputs of the FP8 attention variant for workload ``w``: q and k (the call's
+    own and the cached keys) as E4M3 codes standing for already rotated operands
+    (multipliers E4M3_Q_SCALE, E4M3_K_SCALE), v and cached v as bf16 bits.  Same
+    shapes, K x 3 heads and draw order as ``make_inputs``; cache rows past the
+    cached tokens hold NaN codes."""
+    rng = np.random.default_rng(seed)
+    lay = w.layout
+    B, H, D = lay.batch, w.heads, w.head_dim
+    heads_x = boosted_heads(rng, H, w.k_boost_frac)
+    kscale = np.ones(H, dtype=np.float32)
+    kscale[heads_x] = w.k_boost
+    out: Dict[str, np.ndarray] = {"boosted_heads": heads_x}
+    out["q8"] = normal_e4m3(rng, (B, lay.q_len, H, D), E4M3_Q_SCALE)
+    out["k8"] = normal_e4m3(rng, (B, lay.self_kv_len, H, D), E4M3_K_SCALE, kscale)
+    out["v"] = normal_bf16(rng, (B, lay.self_kv_len, H, D))
+    if lay.mode == MODE_DECODE:
+        n = w.cache_tokens
+        cap = n if cache_capacity is None else cache_capacity
+        ck = np.full((B, cap, H, D), 0x7F, dtype=np.uint8)
+        cv = np.full((B, cap, H, D), 0x7FC1, dtype=np.uint16)
+        ck[:, :n] = normal_e4m3(rng, (B, n, H, D), E4M3_K_SCALE, kscale)
+        cv[:, :n] = normal_bf16(rng, (B, n, H, D))
+        out["cache_k8"], out["cache_v"] = ck, cv
+    return out
+
+
 def cross_layout(w: Workload) -> Layout:
     """Layout of the cross-attention call of workload ``w`` (one query chunk)."""
     lay = w.layout

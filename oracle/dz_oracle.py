@@ -49,7 +49,9 @@ Readings taken where the pages are silent:
   * cross-attention: one softmax over all condition keys, no rotary, no mask.
 
 Parity pins: see tests/test_oracle.py (brute force, library SDPA, closed forms,
-invariants, golden fixtures).  No function here is "parity unpinned".
+invariants, golden fixtures) and tests/test_oracle_e4m3.py (the E4M3 format
+against torch's float8_e4m3fn, brute force, scale invariance).  No function
+here is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -415,3 +417,68 @@ def kvcache_replace(cache_k: np.ndarray, cache_v: np.ndarray, chunk_index: int,
     a = chunk_index * chunk_len_
     cache_k[:, a:a + chunk_len_] = k
     cache_v[:, a:a + chunk_len_] = v
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) variant of the attention.  The walkthrough's system optimisations
+# section: on Blackwell the authors run parts of the DiT in FP8 / NVFP4 and keep
+# the rotary embedding in higher precision.  Here the scores QK^T take rotated q
+# and k as E4M3 codes with one multiplier per tensor (code = E4M3(x * scale));
+# values, probabilities and the output stay as in the bf16 path.
+#
+# E4M3 (the 8-bit floating-point format with 4 exponent and 3 mantissa bits):
+# sign bit, exponent field e (bias 7), mantissa field m; e = 0 encodes the
+# subnormals m/8 * 2^-6; e = 15 with m = 7 is NaN; there are no infinities, so
+# the largest finite magnitude is 1.75 * 2^8 = 448.
+# ---------------------------------------------------------------------------
+
+def e4m3_value(codes: np.ndarray) -> np.ndarray:
+    """Exact value of E4M3 codes (uint8) as float64; NaN for the two NaN codes."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = c & 7
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def quantize_e4m3(x: np.ndarray, scale: float) -> np.ndarray:
+    """E4M3 codes of float32(x * scale): the product is formed in float32 (round to
+    nearest even), then rounded to the nearest finite E4M3 value, ties to the even
+    code, magnitudes past 448 saturating to 448; the sign is kept (so negative
+    values that round to zero give -0); NaN gives the NaN code."""
+    y = (np.asarray(x, dtype=np.float32) * np.float32(scale)).astype(np.float32)
+    a = np.abs(y.astype(np.float64))
+    grid = e4m3_value(np.arange(127, dtype=np.uint8))  # codes 0..126: 0, ..., 448
+    hi = np.clip(np.searchsorted(grid, a, side="left"), 0, 126)
+    lo = np.clip(hi - 1, 0, 126)
+    d_lo = a - grid[lo]
+    d_hi = grid[hi] - a
+    pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a >= 448.0, 126, pick)
+    code = pick.astype(np.uint8) | (np.signbit(y).astype(np.uint8) << 7)
+    return np.where(np.isnan(y), np.uint8(0x7F) | (np.signbit(y).astype(np.uint8) << 7),
+                    code).astype(np.uint8)
+
+
+def chunk_attn_forward_e4m3(q8: np.ndarray, k8: np.ndarray, v_bits: np.ndarray, mode: int,
+                            F: int, gh: int, gw: int, n_action: int, num_chunks: int,
+                            q_scale: float, k_scale: float, kv_len: int = 0,
+                            cache_k8: Optional[np.ndarray] = None,
+                            cache_v_bits: Optional[np.ndarray] = None, cache_len: int = 0,
+                            heads: Optional[slice] = None) -> np.ndarray:
+    """dz_chunk_attn_forward_e4m3: q and k (and the cache keys) arrive rotated, as E4M3
+    codes with multipliers q_scale and k_scale; each operand is its code's value
+    divided by its multiplier.  No rotary is applied.  Returns float64 [B, Sq, H, D]."""
+    L = chunk_len(F, gh, gw, n_action)
+    hs = slice(None) if heads is None else heads
+    q = e4m3_value(q8[:, :, hs, :]) / q_scale
+    k = e4m3_value(k8[:, :, hs, :]) / k_scale
+    v = widen_bf16(v_bits[:, :, hs, :])
+    if mode == DECODE and cache_len > 0:
+        k = np.concatenate([e4m3_value(cache_k8[:, :cache_len, hs, :]) / k_scale, k], axis=1)
+        v = np.concatenate([widen_bf16(cache_v_bits[:, :cache_len, hs, :]), v], axis=1)
+    vis = visibility(mode, L, num_chunks, cache_len=cache_len, kv_len=kv_len)
+    assert vis.shape == (q.shape[1], k.shape[1]), (vis.shape, q.shape, k.shape)
+    return masked_attention(q, k, v, vis)

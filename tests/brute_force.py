@@ -104,8 +104,10 @@ def may_attend(mode: int, qtok, ktok) -> bool:
 
 def attention(q, k, v, mode: int, L: int, num_chunks: int, F: int, gh: int, gw: int,
               t_offset: int = 0, cache_k=None, cache_v=None, cache_len: int = 0,
-              kv_len: int = 0, pairs=(22, 21, 21), base: float = 10000.0):
-    """q, k, v: nested lists [B][S][H][D] of floats. Returns [B][Sq][H][D]."""
+              kv_len: int = 0, pairs=(22, 21, 21), base: float = 10000.0,
+              rotate: bool = True):
+    """q, k, v: nested lists [B][S][H][D] of floats. Returns [B][Sq][H][D].
+    With ``rotate`` false, q and k are taken as already rotated."""
     queries, keys = token_table(mode, L, num_chunks, F, gh, gw, t_offset, cache_len, kv_len)
     B, H, D = len(q), len(q[0][0]), len(q[0][0][0])
     out = [[[None] * H for _ in range(len(queries))] for _ in range(B)]
@@ -118,16 +120,18 @@ def attention(q, k, v, mode: int, L: int, num_chunks: int, F: int, gh: int, gw: 
                     kvecs.append(list(cache_k[b][s][h]))
                     vvecs.append(list(cache_v[b][s][h]))
                 for s in range(L):
-                    kvecs.append(rotate_token(k[b][s][h], keys[cache_len + s][2], pairs, base))
+                    kvecs.append(rotate_token(k[b][s][h], keys[cache_len + s][2], pairs, base)
+                                 if rotate else list(k[b][s][h]))
                     vvecs.append(list(v[b][s][h]))
             else:
                 for s, tok in enumerate(keys):
                     kk = k[b][s][h]
-                    kvecs.append(list(kk) if tok[2] is None else rotate_token(kk, tok[2], pairs, base))
+                    kvecs.append(list(kk) if tok[2] is None or not rotate
+                                 else rotate_token(kk, tok[2], pairs, base))
                     vvecs.append(list(v[b][s][h]))
             for i, qt in enumerate(queries):
                 qq = q[b][i][h]
-                qv = list(qq) if qt[2] is None else rotate_token(qq, qt[2], pairs, base)
+                qv = list(qq) if qt[2] is None or not rotate else rotate_token(qq, qt[2], pairs, base)
                 scores = []
                 for j, kt in enumerate(keys):
                     if may_attend(mode, qt, kt):
