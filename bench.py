@@ -607,6 +607,61 @@ def extra_workload_block(wl: int, dev, stream, steps: int, peak_tf: float, peak_
     return res
 
 
+E4M3_WORKLOADS = (1, 2, 3, 4, 5)
+
+
+def e4m3_block(wl: int, dev, stream, steps: int, peak_tf: float):
+    """The FP8 variant (dz_chunk_attn_forward_e4m3) on workload wl's self-attention:
+    q, k and cached k as rotated E4M3 codes, v bf16, timed like the headline (graphs of
+    calls cycling input sets above L2, CUDA events on the launching stream).  Its QK^T
+    runs at the E4M3 rate and PV at the bf16 rate, so the contraction's peak is taken
+    as the bf16 peak x 4/3 (half the FLOPs at twice the rate)."""
+    import torch
+    from causal_video_diffusion_rope_b200 import dz
+    w = synth.WORKLOADS[wl]
+    lay = w.layout
+    B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
+    keys = w.cache_tokens + lay.self_kv_len
+    set_bytes = B * H * D * (lay.q_len * (1 + 2) + keys * (1 + 2))
+    n_sets = min(4, max(2, int(math.ceil(3 * L2_BYTES / set_bytes))))
+    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len))
+    dl = dz.layout_from(lay)
+    sets = []
+    for i in range(n_sets):
+        inp = synth.make_inputs_e4m3(w, 3000 + 100 * wl + i)
+        s = {"q8": torch.from_numpy(inp["q8"]).to(dev), "k8": torch.from_numpy(inp["k8"]).to(dev),
+             "v": torch.from_numpy(inp["v"].view(np.int16)).to(dev).view(torch.bfloat16),
+             "out": torch.empty((B, lay.q_len, H, D), dtype=torch.bfloat16, device=dev),
+             "cache": None}
+        if "cache_k8" in inp:
+            s["ck8"] = torch.from_numpy(inp["cache_k8"]).to(dev)
+            s["cv"] = torch.from_numpy(inp["cache_v"].view(np.int16)).to(dev).view(torch.bfloat16)
+            s["cache"] = dz.make_cache(s["ck8"], s["cv"], B, w.cache_tokens, w.cache_tokens, L)
+        sets.append(s)
+
+    def call(i):
+        s = sets[i % n_sets]
+        dz.dz_chunk_attn_forward_e4m3(h, s["q8"], s["k8"], s["v"], s["cache"], dl,
+                                      synth.E4M3_Q_SCALE, synth.E4M3_K_SCALE, s["out"], stream)
+
+    n = max(20, min(steps, 240))
+    ms, _ = time_graph(stream, call, n, 3, 1, dev)
+    dz.dz_attn_sync_status(h, stream)
+    dz.dz_attn_destroy(h)
+    us = 1e3 * ms / n
+    tf = self_flops(w) / (us * 1e-6) / 1e12
+    mixed = peak_tf * 4.0 / 3.0
+    res = {"workload": w.name, "what": "attention kernel on E4M3 q, k (rotated, quantised "
+           "beforehand), bf16 v", "calls": n,
+           "l2": f"{n_sets} input sets of {set_bytes / 2**20:.0f} MiB cycle",
+           "us_per_call": round(us, 3), "tflops": round(tf, 2), "flop_per_call": self_flops(w),
+           "frac_of_bf16_peak": round(tf / peak_tf, 4), "mixed_peak": round(mixed, 1),
+           "frac": round(tf / mixed, 4)}
+    sets.clear()
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_attention(args, rank: int, world: int, local_rank: int):
     """The headline: K steps of the attention call on this rank, timed with CUDA events
     (max over ranks); then the end-to-end leg through the same C-ABI call with host
@@ -665,6 +720,8 @@ def run_attention(args, rank: int, world: int, local_rank: int):
         peak_tf, peak_hbm, _ = measured_peaks()
         extra = [extra_workload_block(x, dev, stream, args.steps, peak_tf, peak_hbm, rotation_pass)
                  for x in EXTRA_WORKLOADS if x != args.workload]
+        extra = {"bf16": extra, "e4m3": [e4m3_block(x, dev, stream, args.steps, peak_tf)
+                                         for x in E4M3_WORKLOADS]}
     return ms_per_step, tflops_total, clocks, e2e, ran, extra
 
 
@@ -1045,7 +1102,8 @@ def rank_main(argv) -> None:
             "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": args.steps * launches_per_step(w, rotation_pass), "clocks": clocks}
     if extra is not None:
-        line["workloads"] = extra
+        line["workloads"] = extra["bf16"]
+        line["e4m3"] = extra["e4m3"]
     print(json.dumps(line), flush=True)
 
 

@@ -47,17 +47,20 @@ dz_status cuda_status(cudaError_t e, const char* where = "") {
 }
 
 // 4-D view [B][rows][H][128] of a bf16 BSHD buffer whose batch stride is
-// `rows_alloc` tokens; 64 x 1 x 128 x 1 boxes with 128-byte swizzle.
+// `rows_alloc` tokens; 64 x 1 x 128 x 1 boxes with 128-byte swizzle.  With `bytes`,
+// the buffer holds one-byte (E4M3) elements and the boxes are 128 x 1 x 128 x 1.
 dz_status make_map(const dz_attn* a, CUtensorMap* m, const void* base, int B, int rows,
-                   int rows_alloc, int H) {
+                   int rows_alloc, int H, bool bytes = false) {
+  const cuuint64_t esize = bytes ? 1 : 2;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(dz::HEAD_DIM), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(B)};
-  const cuuint64_t row_bytes = static_cast<cuuint64_t>(H) * dz::HEAD_DIM * 2;
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(dz::HEAD_DIM) * 2, row_bytes,
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(H) * dz::HEAD_DIM * esize;
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(dz::HEAD_DIM) * esize, row_bytes,
                                  row_bytes * static_cast<cuuint64_t>(rows_alloc)};
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(dz::TILE_N), 1};
+  const cuuint32_t box[4] = {bytes ? 128u : 64u, 1, static_cast<cuuint32_t>(dz::TILE_N), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = a->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+  CUresult r = a->encode(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                         4, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -396,12 +399,19 @@ dz_status dz_rope3d(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
 
 // The attention call; with lse != null (training form) it also writes each query
 // row's log2-domain softmax normaliser.
+// e4m3: null for bf16 q and k; else {q multiplier, k multiplier} of E4M3 q, k and
+// cache k, which are then taken as rotated.
 static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const void* v,
                               const dz_kvcache* cache, const dz_chunk_layout* l, void* out,
-                              float* lse, void* stream) {
+                              float* lse, void* stream, const float* e4m3 = nullptr) {
   if (!a || !q || !k || !v || !l || !out) return DZ_ERR_INVALID_ARG;
+  if (e4m3) {
+    for (int i = 0; i < 2; ++i)
+      if (!(e4m3[i] > 0.f) || !std::isfinite(e4m3[i])) return DZ_ERR_INVALID_ARG;
+    if (lse) return DZ_ERR_UNSUPPORTED;
+  }
   // inputs already rotated: the flag is taken off a local copy of the layout
-  const bool given_rotated = (l->mode & DZ_MODE_ROTATED) != 0;
+  const bool given_rotated = (l->mode & DZ_MODE_ROTATED) != 0 || e4m3 != nullptr;
   dz_chunk_layout l_plain = *l;
   l_plain.mode &= ~DZ_MODE_ROTATED;
   l = &l_plain;
@@ -455,6 +465,8 @@ static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const v
 
   dz::AttnLaunch p;
   std::memset(&p, 0, sizeof(p));
+  p.e4m3 = e4m3 ? 1 : 0;
+  p.qk_scale = e4m3 ? 1.0 / (static_cast<double>(e4m3[0]) * e4m3[1]) : 1.0;
   p.sched.mode = l->mode;
   p.sched.Sq = static_cast<int>(Sq);
   p.sched.Sk = static_cast<int>(Sk);
@@ -521,11 +533,13 @@ static dz_status attn_forward(dz_attn_t a, const void* q, const void* k, const v
   p.out_elems -= g_test_out_shrink;
 #endif
 
-  st = make_map(a, &p.tm_q, q_att, l->batch, static_cast<int>(Sq), static_cast<int>(Sq), H);
-  if (st == DZ_OK) st = make_map(a, &p.tm_k, k_att, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
+  const bool f8 = e4m3 != nullptr;
+  st = make_map(a, &p.tm_q, q_att, l->batch, static_cast<int>(Sq), static_cast<int>(Sq), H, f8);
+  if (st == DZ_OK)
+    st = make_map(a, &p.tm_k, k_att, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H, f8);
   if (st == DZ_OK) st = make_map(a, &p.tm_v, v, l->batch, static_cast<int>(Sk), static_cast<int>(Sk), H);
   if (st == DZ_OK && cache_len > 0) {
-    st = make_map(a, &p.tm_ck, cache->k, l->batch, cache_len, cache->capacity_tokens, H);
+    st = make_map(a, &p.tm_ck, cache->k, l->batch, cache_len, cache->capacity_tokens, H, f8);
     if (st == DZ_OK)
       st = make_map(a, &p.tm_cv, cache->v, l->batch, cache_len, cache->capacity_tokens, H);
   }
@@ -544,6 +558,25 @@ dz_status dz_chunk_attn_forward(dz_attn_t a, const void* q, const void* k, const
                                 const dz_kvcache* cache, const dz_chunk_layout* l, void* out,
                                 void* stream) {
   return attn_forward(a, q, k, v, cache, l, out, nullptr, stream);
+}
+
+dz_status dz_chunk_attn_forward_e4m3(dz_attn_t a, const void* q8, const void* k8, const void* v,
+                                     const dz_kvcache* cache, const dz_chunk_layout* l,
+                                     float q_scale, float k_scale, void* out, void* stream) {
+  const float sc[2] = {q_scale, k_scale};
+  return attn_forward(a, q8, k8, v, cache, l, out, nullptr, stream, sc);
+}
+
+dz_status dz_quantize_e4m3(dz_attn_t a, const void* x, void* y, int64_t n, float scale,
+                           void* stream) {
+  if (!a || !x || !y || n < 0) return DZ_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return DZ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return DZ_ERR_ALIGNMENT;
+  if (n == 0) return DZ_OK;
+  return cuda_status(dz::launch_quantize_e4m3(static_cast<const __nv_bfloat16*>(x),
+                                              static_cast<uint8_t*>(y), n, scale,
+                                              static_cast<cudaStream_t>(stream)),
+                     "quantize launch");
 }
 
 dz_status dz_chunk_attn_forward_lse(dz_attn_t a, const void* q, const void* k, const void* v,

@@ -40,6 +40,12 @@
 // publishes fp32 partial (O, m, l) to the workspace, and the last one merges
 // them into its own O in TMEM.  With the call's q and own k rotated once into a
 // workspace beforehand (or given rotated), the rotary gate only passes tiles on.
+//
+// E4M3 variant (second template argument): q and k arrive rotated as E4M3 codes (one
+// byte per element, one 128-byte swizzle row per token, 16 KiB per tile in the first
+// half of each Q/K slot) and QK^T runs as kind::f8f6f4 products of K = 32; the
+// multipliers of q and k are folded into the softmax scale.  V, P, O and the output
+// are as in the bf16 kernel.
 #include <type_traits>
 
 #include "dz_internal.cuh"
@@ -58,6 +64,7 @@ constexpr int ROPE_THREADS = (WARP_SOFT - WARP_ROPE) * 32;
 constexpr int KV_STAGES = 2;
 constexpr int TILE_BYTES = TILE_M * HEAD_DIM * 2;  // 32 KiB
 constexpr int HALF_BYTES = TILE_BYTES / 2;         // 64 dims x 128 rows
+constexpr int TILE_BYTES_E4M3 = TILE_M * HEAD_DIM;  // 16 KiB: 128 one-byte dims x 128 rows
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 // Registers per thread: the kernel is compiled for LAUNCH_REGS (3 warps per SM
@@ -401,7 +408,7 @@ __device__ __forceinline__ int cta_of(const unsigned* tb, int G, unsigned x) {
 
 }  // namespace
 
-template <class P>
+template <class P, bool F8>
 __global__ void __launch_bounds__(NTHREADS, 1)
     chunk_attn_kernel(const __grid_constant__ P p) {
   constexpr bool kWaves = std::is_same<P, AttnParamsWaves>::value;
@@ -528,11 +535,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const int b = sg.bh / p.H, h = sg.bh - (sg.bh / p.H) * p.H;
         // Q of this segment: the previous segment's last QK products must be done
         if (seg_i > 0 && !mbar_wait(&bar[B_Q_EMPTY], (seg_i - 1) & 1, abort_flag, p.status)) break;
-        mbar_expect_tx(&bar[B_Q_FULL], Q_TILES * TILE_BYTES);
+        mbar_expect_tx(&bar[B_Q_FULL], Q_TILES * (F8 ? TILE_BYTES_E4M3 : TILE_BYTES));
         for (int q = 0; q < Q_TILES; ++q) {
           const int row = sg.qg * Q_GROUP + q * TILE_M;
           tma_load_4d(sQ + q * TILE_BYTES, &p.tm_q, &bar[B_Q_FULL], 0, h, row, b);
-          tma_load_4d(sQ + q * TILE_BYTES + HALF_BYTES, &p.tm_q, &bar[B_Q_FULL], 64, h, row, b);
+          if constexpr (!F8)
+            tma_load_4d(sQ + q * TILE_BYTES + HALF_BYTES, &p.tm_q, &bar[B_Q_FULL], 64, h, row, b);
         }
         ++q_loads;
         for (int i = 0; i < sg.n; ++i) {
@@ -543,9 +551,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const CUtensorMap* mv = kt.cache ? &p.tm_cv : &p.tm_v;
           if (!mbar_wait(&bar[B_K_EMPTY + st], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
           uint64_t* kb = &bar[(kt.rope ? B_K_RAW : B_K_FULL) + st];
-          mbar_expect_tx(kb, TILE_BYTES);
+          mbar_expect_tx(kb, F8 ? TILE_BYTES_E4M3 : TILE_BYTES);
           tma_load_4d(sK + st * TILE_BYTES, mk, kb, 0, h, kt.row0, b);
-          tma_load_4d(sK + st * TILE_BYTES + HALF_BYTES, mk, kb, 64, h, kt.row0, b);
+          if constexpr (!F8) tma_load_4d(sK + st * TILE_BYTES + HALF_BYTES, mk, kb, 64, h, kt.row0, b);
           if (kt.rope) ++kr_cnt[st]; else ++kf_cnt[st];
           ++k_iss;
           // the V stage held V(t - 2), whose products were issued before QK(t - 1): the
@@ -577,7 +585,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp == WARP_MMA) {
     // ======================= tcgen05 issuer =======================
     if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16(TILE_M, TILE_N, false);
+      const uint32_t idesc_qk = F8 ? idesc_e4m3(TILE_M, TILE_N) : idesc_bf16(TILE_M, TILE_N, false);
       const uint32_t idesc_pv = idesc_bf16(TILE_M, HEAD_DIM, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       // descriptors: only the low word (start address) changes between the K-steps
@@ -585,10 +593,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto issue_qk = [&](int q, int st) {
         const uint32_t a0 = q_lo + ((q * TILE_BYTES) >> 4), b0 = k_lo + ((st * TILE_BYTES) >> 4);
         const uint32_t d = tmem + q * TILE_N;
+        if constexpr (F8) {
+          // one 128-byte row per token: the four K = 32 steps walk along it
 #pragma unroll
-        for (int kk = 0; kk < HEAD_DIM / 16; ++kk) {
-          const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
-          mma_ss(d, desc_join(a0 + off), desc_join(b0 + off), idesc_qk, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < HEAD_DIM / 32; ++kk) {
+            const uint32_t off = (kk * 32) >> 4;
+            mma_ss_e4m3(d, desc_join(a0 + off), desc_join(b0 + off), idesc_qk, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < HEAD_DIM / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * HALF_BYTES + (kk & 3) * 32) >> 4;
+            mma_ss(d, desc_join(a0 + off), desc_join(b0 + off), idesc_qk, kk > 0 ? 1u : 0u);
+          }
         }
       };
       auto issue_pv = [&](int q, int st, bool acc) {
@@ -1024,7 +1041,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-template <class P>
+template <class P, bool F8>
 static cudaError_t prepare_kernel() {
   static bool attr_set[64] = {};
   int dev = 0;
@@ -1032,10 +1049,10 @@ static cudaError_t prepare_kernel() {
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
     // the warpgroup register split assumes exactly LAUNCH_REGS registers per thread
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_attn_kernel<P>);
+    cudaError_t e = cudaFuncGetAttributes(&fa, chunk_attn_kernel<P, F8>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(chunk_attn_kernel<P>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(chunk_attn_kernel<P, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
@@ -1070,27 +1087,35 @@ static void fill_params(AttnParams& p, const AttnLaunch& a) {
   p.stage_nt = a.stage_nt;
   p.W = static_cast<unsigned>(a.W);
   p.G = a.grid;
-  p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(HEAD_DIM)) *
+                                    a.qk_scale);
 }
 
-cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
+template <bool F8>
+static cudaError_t launch_variant(const AttnLaunch& a, cudaStream_t stream) {
   // the plain split computes c * W / G in 32 bits; past that the ranges go explicitly
   if (a.waves > 0 || a.W * (a.grid + 1LL) >= (1LL << 31)) {
-    cudaError_t e = prepare_kernel<AttnParamsWaves>();
+    cudaError_t e = prepare_kernel<AttnParamsWaves, F8>();
     if (e != cudaSuccess) return e;
     AttnParamsWaves p;
     fill_params(p, a);
     p.waves = a.waves;
     for (int c = 0; c <= a.grid; ++c) p.tb[c] = a.tb[c];
-    chunk_attn_kernel<AttnParamsWaves><<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    chunk_attn_kernel<AttnParamsWaves, F8><<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
   } else {
-    cudaError_t e = prepare_kernel<AttnParams>();
+    cudaError_t e = prepare_kernel<AttnParams, F8>();
     if (e != cudaSuccess) return e;
     AttnParams p;
     fill_params(p, a);
-    chunk_attn_kernel<AttnParams><<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
+    chunk_attn_kernel<AttnParams, F8><<<a.grid, NTHREADS, SMEM_BYTES, stream>>>(p);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_attention(const AttnLaunch& a, cudaStream_t stream) {
+  // E4M3 operands arrive rotated: the kernel would not rotate them
+  if (a.e4m3 && (a.rope_q || a.rope_k)) return cudaErrorInvalidValue;
+  return a.e4m3 ? launch_variant<true>(a, stream) : launch_variant<false>(a, stream);
 }
 
 }  // namespace dz

@@ -189,6 +189,10 @@ cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const Chu
                           int first_chunk, const RopeTables& r, int* status, cudaStream_t stream,
                           const void* x1 = nullptr, void* y1 = nullptr, int period = 0);
 
+// y[0:n] = E4M3 codes of x[0:n] * scale (round to nearest even, saturating at 448).
+cudaError_t launch_quantize_e4m3(const __nv_bfloat16* x, uint8_t* y, long long n, float scale,
+                                 cudaStream_t stream);
+
 struct AttnLaunch {
   CUtensorMap tm_q, tm_k, tm_v, tm_ck, tm_cv;
   void* out;
@@ -218,6 +222,10 @@ struct AttnLaunch {
   int grid;
   int waves;
   unsigned tb[MAX_GRID + 1];
+  // q and k (and cache k) are rotated E4M3 codes rather than bf16; the scores are
+  // multiplied by qk_scale (1 / (q multiplier * k multiplier); 1 for bf16 operands)
+  int e4m3;
+  double qk_scale;
 };
 
 // Schedule of an attention call (see AttnLaunch): fills grid, waves and tb from the

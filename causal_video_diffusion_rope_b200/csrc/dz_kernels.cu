@@ -1,5 +1,7 @@
 // Bandwidth-bound kernels: KV-cache append/replace (a 16-byte vectorised
-// copy) and the standalone 3D rotary embedding.
+// copy), the standalone 3D rotary embedding and the E4M3 quantisation.
+#include <cuda_fp8.h>
+
 #include "dz_internal.cuh"
 #include "dz_ptx.cuh"
 
@@ -117,6 +119,62 @@ cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const Chu
   rope3d_kernel<<<grid, ROPE_BLOCK, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
                                           static_cast<const uint4*>(x1), static_cast<uint4*>(y1),
                                           S, H, g, first_chunk, period, r, status);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// E4M3 quantisation: y[i] = E4M3(float(x[i]) * scale), rounded to nearest even with
+// magnitudes past 448 saturating (the FP8 operands of the attention's QK^T).  Each
+// thread turns 16 bf16 values (two 16-byte loads) into one 16-byte store; the last
+// n % 16 elements go one per thread.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3x4(uint32_t lo2, uint32_t hi2, float scale) {
+  const float2 a = make_float2(__fmul_rn(__uint_as_float(lo2 << 16), scale),
+                               __fmul_rn(__uint_as_float(lo2 & 0xffff0000u), scale));
+  const float2 b = make_float2(__fmul_rn(__uint_as_float(hi2 << 16), scale),
+                               __fmul_rn(__uint_as_float(hi2 & 0xffff0000u), scale));
+  const uint32_t pa = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
+  const uint32_t pb = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
+  return pa | (pb << 16);
+}
+
+__global__ void __launch_bounds__(256) quantize_e4m3_kernel(const uint4* __restrict__ x,
+                                                            uint4* __restrict__ y, long long nvec,
+                                                            float scale) {
+  const long long step = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
+       i += step) {
+    const uint4 a = x[2 * i], b = x[2 * i + 1];
+    y[i] = make_uint4(e4m3x4(a.x, a.y, scale), e4m3x4(a.z, a.w, scale), e4m3x4(b.x, b.y, scale),
+                      e4m3x4(b.z, b.w, scale));
+  }
+}
+
+__global__ void quantize_e4m3_tail_kernel(const uint16_t* __restrict__ x, uint8_t* __restrict__ y,
+                                          int n, float scale) {
+  const int i = threadIdx.x;
+  if (i < n) {
+    const float v = __fmul_rn(__uint_as_float(static_cast<uint32_t>(x[i]) << 16), scale);
+    y[i] = static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+  }
+}
+
+cudaError_t launch_quantize_e4m3(const __nv_bfloat16* x, uint8_t* y, long long n, float scale,
+                                 cudaStream_t stream) {
+  const long long nvec = n / 16;
+  if (nvec > 0) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long need = (nvec + 255) / 256;
+    const int blocks = static_cast<int>(need < 8LL * sms ? need : 8LL * sms);
+    quantize_e4m3_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<const uint4*>(x),
+                                                     reinterpret_cast<uint4*>(y), nvec, scale);
+  }
+  const int tail = static_cast<int>(n - nvec * 16);
+  if (tail > 0)
+    quantize_e4m3_tail_kernel<<<1, 32, 0, stream>>>(
+        reinterpret_cast<const uint16_t*>(x) + nvec * 16, y + nvec * 16, tail, scale);
   return cudaGetLastError();
 }
 

@@ -36,7 +36,7 @@ EXPORTS = [
     "dz_attn_create", "dz_attn_destroy", "dz_rope3d", "dz_chunk_attn_forward",
     "dz_kvcache_append", "dz_kvcache_replace", "dz_attn_sync_status", "dz_status_string",
     "dz_chunk_attn_forward_noalloc", "dz_qkv_rope", "dz_chunk_attn_forward_lse",
-    "dz_chunk_attn_backward",
+    "dz_chunk_attn_backward", "dz_chunk_attn_forward_e4m3", "dz_quantize_e4m3",
 ]
 
 
@@ -98,6 +98,10 @@ def bind(lib: ctypes.CDLL) -> ctypes.CDLL:
                                               vp, vp, vp]
     lib.dz_chunk_attn_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp,
                                            ctypes.POINTER(dz_chunk_layout), vp, vp, vp, vp]
+    lib.dz_chunk_attn_forward_e4m3.argtypes = [vp, vp, vp, vp, ctypes.POINTER(dz_kvcache),
+                                               ctypes.POINTER(dz_chunk_layout), ctypes.c_float,
+                                               ctypes.c_float, vp, vp]
+    lib.dz_quantize_e4m3.argtypes = [vp, vp, vp, ctypes.c_int64, ctypes.c_float, vp]
     lib.dz_attn_sync_status.argtypes = [vp, vp]
     lib.dz_status_string.argtypes = [ctypes.c_int]
     lib.dz_status_string.restype = ctypes.c_char_p
@@ -195,6 +199,21 @@ def dz_chunk_attn_forward(handle: int, q, k, v, cache: Optional[dz_kvcache],
     _check(load().dz_chunk_attn_forward(handle, _ptr(q), _ptr(k), _ptr(v), cptr,
                                         ctypes.byref(layout), _ptr(out), _stream(stream)),
            "dz_chunk_attn_forward")
+
+
+def dz_chunk_attn_forward_e4m3(handle: int, q8, k8, v, cache: Optional[dz_kvcache],
+                               layout: dz_chunk_layout, q_scale: float, k_scale: float, out,
+                               stream=None) -> None:
+    cptr = ctypes.byref(cache) if cache is not None else None
+    _check(load().dz_chunk_attn_forward_e4m3(handle, _ptr(q8), _ptr(k8), _ptr(v), cptr,
+                                             ctypes.byref(layout), q_scale, k_scale, _ptr(out),
+                                             _stream(stream)),
+           "dz_chunk_attn_forward_e4m3")
+
+
+def dz_quantize_e4m3(handle: int, x, y, n: int, scale: float, stream=None) -> None:
+    _check(load().dz_quantize_e4m3(handle, _ptr(x), _ptr(y), n, scale, _stream(stream)),
+           "dz_quantize_e4m3")
 
 
 def dz_chunk_attn_forward_noalloc(desc: dz_attn_desc, q, k, v, cache: Optional[dz_kvcache],

@@ -192,6 +192,32 @@ dz_status dz_chunk_attn_forward(dz_attn_t handle, const void* q, const void* k, 
                                 const dz_kvcache* cache, const dz_chunk_layout* layout,
                                 void* out, void* stream);
 
+/* FP8 variant of dz_chunk_attn_forward (the walkthrough of "World Action Models
+ * are Zero-shot Policies", system optimisations: on Blackwell the DiT runs in
+ * FP8 / NVFP4 with the rotary embedding kept in higher precision).  q8, k8 and,
+ * in DECODE, cache->k hold ROTATED q and k as E4M3 codes (one byte per element,
+ * same [B][S][H][128] layout; code = E4M3(x * multiplier), see dz_quantize_e4m3)
+ * with multipliers q_scale and k_scale; v, cache->v and out are bf16 as in
+ * dz_chunk_attn_forward.  Scores = (q8 . k8) / (q_scale * k_scale) / sqrt(128):
+ * QK^T runs on E4M3 operands with fp32 accumulation; softmax, P (bf16), PV and
+ * the output are as in the bf16 path.  No rotation is applied (DZ_MODE_ROTATED
+ * is implied); modes as in dz_chunk_attn_forward.
+ * Errors: as dz_chunk_attn_forward, and DZ_ERR_INVALID_ARG for a multiplier that
+ * is not finite and positive. */
+dz_status dz_chunk_attn_forward_e4m3(dz_attn_t handle, const void* q8, const void* k8,
+                                     const void* v, const dz_kvcache* cache,
+                                     const dz_chunk_layout* layout, float q_scale, float k_scale,
+                                     void* out, void* stream);
+
+/* E4M3 quantisation of n bf16 values: y[i] = E4M3(float(x[i]) * scale), the
+ * product formed in fp32 and rounded to the nearest E4M3 value (ties to even),
+ * magnitudes past 448 saturating to 448, sign kept (-0 for negatives that round
+ * to zero), NaN to a NaN code.  x bf16 [n], y uint8 [n], both 16-byte aligned.
+ * Errors: DZ_ERR_INVALID_ARG (n < 0, scale not finite and positive),
+ * DZ_ERR_ALIGNMENT, DZ_ERR_CUDA. */
+dz_status dz_quantize_e4m3(dz_attn_t handle, const void* x, void* y, int64_t n, float scale,
+                           void* stream);
+
 /* Append one chunk (KV cache of clean chunks: "DreamZero 单卡推理", "架构"
  * table -- the DiT runner keeps the attention KV; "连续请求" -- KV carried
  * across requests).  Copies k, v bf16 [cache->batch][L][H][128]

@@ -83,6 +83,9 @@ def test_calls_reject_null_handle(lib):
         dz.DZ_ERR_INVALID_ARG
     assert lib.dz_chunk_attn_backward(None, 16, 16, 16, 16, 16, 16, ctypes.byref(pre), 16, 16,
                                       16, None) == dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_chunk_attn_forward_e4m3(None, 16, 16, 16, None, ctypes.byref(lay), 64.0, 16.0,
+                                          16, None) == dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_quantize_e4m3(None, 16, 16, 128, 1.0, None) == dz.DZ_ERR_INVALID_ARG
     # a null layout or output pointer is rejected before any handle lookup
     assert lib.dz_chunk_attn_forward_lse(None, 16, 16, 16, None, 16, 16, None) == \
         dz.DZ_ERR_INVALID_ARG
