@@ -129,8 +129,8 @@ def measured_peaks():
 
 def ncu_traffic(workload_name: str):
     """Per-launch DRAM bytes of the attention kernel on a workload from the committed ncu
-    summary (profiles/attn_<workload>.json), or None if there is none or it was taken on
-    different kernel sources."""
+    summary (profiles/attn_<workload>.json; the E4M3 variant's as attn_e4m3_<workload>),
+    or None if there is none or it was taken on different kernel sources."""
     path = os.path.join(ROOT, "profiles", f"attn_{workload_name}.json")
     if not os.path.exists(path):
         return None
@@ -608,58 +608,130 @@ def extra_workload_block(wl: int, dev, stream, steps: int, peak_tf: float, peak_
 
 
 E4M3_WORKLOADS = (1, 2, 3, 4, 5)
+E4M3_METRIC = ("chunk-causal attention with E4M3 QK^T TFLOP/s and % of the B200 mixed "
+               "E4M3/BF16 peak; \u00b5s per DiT-layer attention call")
+
+
+class E4m3Setup:
+    """Handle and input sets of workload w's self-attention in the FP8 variant: q, k and
+    cached k as rotated E4M3 codes (synthetic, multipliers E4M3_Q_SCALE / E4M3_K_SCALE),
+    v bf16; sets cycle so that one pass exceeds the L2."""
+
+    def __init__(self, w: synth.Workload, dev, seed_base: int, max_sets: int = 4):
+        import torch
+        from causal_video_diffusion_rope_b200 import dz
+        self.dz, self.w = dz, w
+        lay = w.layout
+        B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
+        keys = w.cache_tokens + lay.self_kv_len
+        self.set_bytes = B * H * D * (lay.q_len * (1 + 2) + keys * (1 + 2))
+        self.n_sets = min(max_sets, max(2, int(math.ceil(3 * L2_BYTES / self.set_bytes))))
+        self.h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len))
+        self.dl = dz.layout_from(lay)
+        self.sets = []
+        for i in range(self.n_sets):
+            inp = synth.make_inputs_e4m3(w, seed_base + i)
+            st = {"q8": torch.from_numpy(inp["q8"]).to(dev), "k8": torch.from_numpy(inp["k8"]).to(dev),
+                  "v": torch.from_numpy(inp["v"].view(np.int16)).to(dev).view(torch.bfloat16),
+                  "out": torch.empty((B, lay.q_len, H, D), dtype=torch.bfloat16, device=dev),
+                  "cache": None}
+            if "cache_k8" in inp:
+                st["ck8"] = torch.from_numpy(inp["cache_k8"]).to(dev)
+                st["cv"] = torch.from_numpy(inp["cache_v"].view(np.int16)).to(dev).view(torch.bfloat16)
+                st["cache"] = dz.make_cache(st["ck8"], st["cv"], B, w.cache_tokens, w.cache_tokens, L)
+            self.sets.append(st)
+
+    def call(self, i, stream, q8=None, k8=None, v=None, out=None):
+        st = self.sets[i % self.n_sets]
+        self.dz.dz_chunk_attn_forward_e4m3(
+            self.h, st["q8"] if q8 is None else q8, st["k8"] if k8 is None else k8,
+            st["v"] if v is None else v, st["cache"], self.dl, synth.E4M3_Q_SCALE,
+            synth.E4M3_K_SCALE, st["out"] if out is None else out, stream)
+
+    def close(self):
+        self.dz.dz_attn_sync_status(self.h)
+        self.dz.dz_attn_destroy(self.h)
+        self.sets.clear()
 
 
 def e4m3_block(wl: int, dev, stream, steps: int, peak_tf: float):
-    """The FP8 variant (dz_chunk_attn_forward_e4m3) on workload wl's self-attention:
-    q, k and cached k as rotated E4M3 codes, v bf16, timed like the headline (graphs of
-    calls cycling input sets above L2, CUDA events on the launching stream).  Its QK^T
-    runs at the E4M3 rate and PV at the bf16 rate, so the contraction's peak is taken
-    as the bf16 peak x 4/3 (half the FLOPs at twice the rate)."""
+    """The FP8 variant (dz_chunk_attn_forward_e4m3) on workload wl's self-attention,
+    timed like the headline (graphs of calls cycling input sets above L2, CUDA events
+    on the launching stream).  Its QK^T runs at the E4M3 rate and PV at the bf16 rate,
+    so the contraction's peak is taken as the bf16 peak x 4/3 (half the FLOPs at twice
+    the rate)."""
     import torch
-    from causal_video_diffusion_rope_b200 import dz
     w = synth.WORKLOADS[wl]
-    lay = w.layout
-    B, H, D, L = lay.batch, w.heads, w.head_dim, lay.chunk_len
-    keys = w.cache_tokens + lay.self_kv_len
-    set_bytes = B * H * D * (lay.q_len * (1 + 2) + keys * (1 + 2))
-    n_sets = min(4, max(2, int(math.ceil(3 * L2_BYTES / set_bytes))))
-    h = dz.dz_attn_create(dz.make_desc(num_heads=H, max_batch=B, max_q_tokens=lay.q_len))
-    dl = dz.layout_from(lay)
-    sets = []
-    for i in range(n_sets):
-        inp = synth.make_inputs_e4m3(w, 3000 + 100 * wl + i)
-        s = {"q8": torch.from_numpy(inp["q8"]).to(dev), "k8": torch.from_numpy(inp["k8"]).to(dev),
-             "v": torch.from_numpy(inp["v"].view(np.int16)).to(dev).view(torch.bfloat16),
-             "out": torch.empty((B, lay.q_len, H, D), dtype=torch.bfloat16, device=dev),
-             "cache": None}
-        if "cache_k8" in inp:
-            s["ck8"] = torch.from_numpy(inp["cache_k8"]).to(dev)
-            s["cv"] = torch.from_numpy(inp["cache_v"].view(np.int16)).to(dev).view(torch.bfloat16)
-            s["cache"] = dz.make_cache(s["ck8"], s["cv"], B, w.cache_tokens, w.cache_tokens, L)
-        sets.append(s)
-
-    def call(i):
-        s = sets[i % n_sets]
-        dz.dz_chunk_attn_forward_e4m3(h, s["q8"], s["k8"], s["v"], s["cache"], dl,
-                                      synth.E4M3_Q_SCALE, synth.E4M3_K_SCALE, s["out"], stream)
-
+    st = E4m3Setup(w, dev, 3000 + 100 * wl)
     n = max(20, min(steps, 240))
-    ms, _ = time_graph(stream, call, n, 3, 1, dev)
-    dz.dz_attn_sync_status(h, stream)
-    dz.dz_attn_destroy(h)
+    ms, _ = time_graph(stream, lambda i: st.call(i, stream), n, 3, 1, dev)
+    st.close()
     us = 1e3 * ms / n
     tf = self_flops(w) / (us * 1e-6) / 1e12
     mixed = peak_tf * 4.0 / 3.0
     res = {"workload": w.name, "what": "attention kernel on E4M3 q, k (rotated, quantised "
            "beforehand), bf16 v", "calls": n,
-           "l2": f"{n_sets} input sets of {set_bytes / 2**20:.0f} MiB cycle",
+           "l2": f"{st.n_sets} input sets of {st.set_bytes / 2**20:.0f} MiB cycle",
            "us_per_call": round(us, 3), "tflops": round(tf, 2), "flop_per_call": self_flops(w),
            "frac_of_bf16_peak": round(tf / peak_tf, 4), "mixed_peak": round(mixed, 1),
-           "frac": round(tf / mixed, 4)}
-    sets.clear()
+           "frac": round(tf / mixed, 4), "traffic": ncu_traffic("e4m3_" + w.name)}
+    del st
     torch.cuda.empty_cache()
     return res
+
+
+def run_e4m3(args, rank: int, world: int, local_rank: int, config: dict):
+    """The FP8 variant as the headline: K calls of dz_chunk_attn_forward_e4m3 on the
+    workload's self-attention (E4M3 q, k and cached k; bf16 v), then the end-to-end leg
+    with q8, k8, v copied in from pinned host memory and out copied back."""
+    import torch
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = synth.WORKLOADS[args.workload]
+    st = E4m3Setup(w, dev, 3000 + 1000 * rank)
+    stream = torch.cuda.Stream(device=dev)
+    sampler = ClockSampler(gpu_id(local_rank))
+    ms, clocks = time_graph(stream, lambda i: st.call(i, stream), args.steps, max(args.warmup, 3),
+                            world, dev, sampler)
+    st.dz.dz_attn_sync_status(st.h, stream)
+    ms_per_step = ms / args.steps
+    fl = self_flops(w)
+    tf = fl / (ms_per_step * 1e-3) / 1e12
+    s0 = st.sets[0]
+
+    def e2e_call(di, do):
+        st.call(0, stream, di["q8"], di["k8"], di["v"], do["out"])
+
+    e2e = e2e_pipelined(dev, stream, {k: s0[k] for k in ("q8", "k8", "v")}, {"out": s0["out"]},
+                        e2e_call, max(3, min(args.steps, 200)), world)
+    e2e["value"] = round(job_throughput(fl, e2e.pop("steps_done"), world, e2e.pop("ms")), 3)
+    n_sets, set_bytes = st.n_sets, st.set_bytes
+    st.close()
+    if rank != 0:
+        return
+    peak_tf, _, peak_kind = measured_peaks()
+    mixed = peak_tf * 4.0 / 3.0
+    line = {"metric": E4M3_METRIC, "value": round(tf * world, 3), "unit": "TFLOP/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6), "us_per_call": round(ms_per_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 q/k, bf16 v/p/out, fp32 accumulation",
+            "data": "synthetic (E4M3 codes of N(0,1) q, k; N(0,1) bf16 v)",
+            "config": dict(config, op="attention_e4m3", q_scale=synth.E4M3_Q_SCALE,
+                           k_scale=synth.E4M3_K_SCALE,
+                           l2=f"inputs cycle through {n_sets} sets "
+                              f"({n_sets * set_bytes / 2**20:.0f} MiB > 126 MB L2)",
+                           parallelism=f"dp{world} (independent replicas of the call)"),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 2), "peak": round(mixed, 1),
+                         "unit": "TFLOP/s", "frac": round(tf / mixed, 4),
+                         "traffic": ncu_traffic("e4m3_" + w.name),
+                         "peak_kind": f"{peak_kind} bf16 (burst) x 4/3: QK^T at the E4M3 rate "
+                                      "(2x bf16), PV at the bf16 rate",
+                         "frac_of_bf16_peak": round(tf / peak_tf, 4),
+                         "kernel": "chunk_attn_kernel (E4M3 instantiation)",
+                         "kernel_us": round(ms_per_step * 1e3, 3)},
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks}
+    print(json.dumps(line), flush=True)
 
 
 def run_attention(args, rank: int, world: int, local_rank: int):
@@ -995,10 +1067,11 @@ def parse_args(argv):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0,
                     help="seconds of oracle CPU work for the cpu_baseline field")
-    ap.add_argument("--op", default="attn", choices=["attn", "qkv", "bwd", "cache"],
+    ap.add_argument("--op", default="attn", choices=["attn", "qkv", "bwd", "cache", "e4m3"],
                     help="attn: the chunk-causal attention call; qkv: the fused projection; "
                          "bwd: the backward of a prefill / teacher-forcing call; "
-                         "cache: the KV-cache chunk replace")
+                         "cache: the KV-cache chunk replace; e4m3: the attention call with "
+                         "E4M3 q and k")
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD,
                     choices=range(len(synth.WORKLOADS)),
                     help="workload index (default: the single-layer inference step)")
@@ -1045,9 +1118,9 @@ def rank_main(argv) -> None:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        if args.op in ("qkv", "bwd", "cache"):
-            {"qkv": run_qkv, "bwd": run_bwd, "cache": run_cache}[args.op](args, rank, world,
-                                                                         local_rank, config)
+        if args.op in ("qkv", "bwd", "cache", "e4m3"):
+            {"qkv": run_qkv, "bwd": run_bwd, "cache": run_cache,
+             "e4m3": run_e4m3}[args.op](args, rank, world, local_rank, config)
             return
         cpu = None
         if rank == 0 and world == 1 and args.cpu_budget > 0:
