@@ -26,6 +26,9 @@
 // thread writes its bf16 operands over its own fp32 columns, so a half's operand
 // occupies columns [0, 16) and [32, 48) of its region (see mma_tmem_a64).  The rotation back (R^T) and the 1/sqrt(128) are applied to the fp32
 // accumulators in the epilogue.
+#include <algorithm>
+#include <vector>
+
 #include "dz_ops.cuh"
 #include "dz_ptx.cuh"
 
@@ -59,6 +62,10 @@ enum {
 };
 static_assert(BB_COUNT * 8 <= 256, "barrier area");
 
+// Tiles per (batch, head) whose launch order the host can sort (larger calls keep
+// the natural order).
+constexpr int BWD_ORDER_MAX = 512;
+
 struct __align__(64) BwdParams {
   CUtensorMap tm_q, tm_k, tm_v, tm_do;  // rotated q, rotated k, v, dO: (128, H, S, B)
   const float* lse;                      // [B][H][S], log2 domain
@@ -71,10 +78,31 @@ struct __align__(64) BwdParams {
   int period;                            // TF: N*L (noisy tokens sit at clean positions)
   float scale_log2, scale;
   int* status;
+  // Launch order: CTAs go out in groups of head_group (batch, head) pairs; inside a
+  // group, rank r of the tiles (heaviest first: order_q for the dQ kernel, order_k for
+  // dK/dV) for every pair of the group, then rank r + 1.  The pairs of a group share
+  // their streamed tiles through L2, and the lightest tiles come last.
+  int head_group, use_order;
+  uint16_t order_q[BWD_ORDER_MAX], order_k[BWD_ORDER_MAX];
 };
 
+// (batch * H + head, tile) of this CTA under the launch order above.
+__device__ __forceinline__ void bwd_unit(const BwdParams& p, const uint16_t* order, int& bh,
+                                         int& tile) {
+  const int BH = p.B * p.H;
+  const int G = p.head_group;
+  const int per = G * p.n_tiles;
+  const int grp = static_cast<int>(blockIdx.x) / per;
+  const int g0 = grp * G;
+  const int gs = min(G, BH - g0);
+  const int rem = static_cast<int>(blockIdx.x) - grp * per;
+  const int rank = rem / gs;
+  bh = g0 + (rem - rank * gs);
+  tile = p.use_order ? static_cast<int>(order[rank]) : rank;
+}
+
 // Visible keys of query s: [a0, a1) and [b0, b1).
-__device__ __forceinline__ void q_keys(const BwdParams& p, int s, int& a0, int& a1, int& b0,
+__host__ __device__ __forceinline__ void q_keys(const BwdParams& p, int s, int& a0, int& a1, int& b0,
                                        int& b1) {
   const int c = s / p.L;
   a0 = 0;
@@ -106,7 +134,7 @@ __device__ __forceinline__ void k_queries(const BwdParams& p, int j, int& a0, in
 }
 
 // Does any query of tile qt see any key of tile kt?
-__device__ __forceinline__ bool pair_visible(const BwdParams& p, int qt, int kt) {
+__host__ __device__ __forceinline__ bool pair_visible(const BwdParams& p, int qt, int kt) {
   const int q0 = qt * BT, q1 = min(q0 + BT, p.S);
   const int k0 = kt * BT, k1 = min(k0 + BT, p.S);
   for (int c = q0 / p.L; c <= (q1 - 1) / p.L; ++c) {
@@ -217,8 +245,8 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dq_kernel(const __grid_consta
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + DQ_SM_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + DQ_SM_MISC + 4);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x % p.n_tiles;
-  const int bh = blockIdx.x / p.n_tiles;
+  int bh, qt;
+  bwd_unit(p, p.order_q, bh, qt);
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int q0 = qt * BT;
 
@@ -437,8 +465,8 @@ __global__ void __launch_bounds__(BTHREADS, 1) bwd_dkv_kernel(const __grid_const
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + BSM_MISC + 4);
   float* sm_vec = reinterpret_cast<float*>(smem + BSM_VEC);  // [2 buffers][lse 128 | D 128]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kt = blockIdx.x % p.n_tiles;
-  const int bh = blockIdx.x / p.n_tiles;
+  int bh, kt;
+  bwd_unit(p, p.order_k, bh, kt);
   const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
   const int k0 = kt * BT;
 
@@ -711,6 +739,29 @@ cudaError_t launch_backward(const BwdLaunch& a, cudaStream_t stream) {
   p.scale = 1.f / sqrtf(static_cast<float>(HEAD_DIM));
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HEAD_DIM));
   p.status = a.status;
+  // launch order: heaviest tiles first inside groups of (batch, head) pairs whose
+  // streamed tiles (2 x S x 256 bytes per pair) fill about a third of the L2
+  const long long pair_bytes = 2LL * a.S * HEAD_DIM * 2;
+  const long long g = (40LL << 20) / (pair_bytes > 0 ? pair_bytes : 1);
+  p.head_group = static_cast<int>(g < 1 ? 1 : (g > a.B * a.H ? a.B * a.H : g));
+  p.use_order = p.n_tiles <= BWD_ORDER_MAX ? 1 : 0;
+  if (p.use_order) {
+    std::vector<int> nq(p.n_tiles, 0), nk(p.n_tiles, 0);
+    for (int qt = 0; qt < p.n_tiles; ++qt)
+      for (int kt = 0; kt < p.n_tiles; ++kt)
+        if (pair_visible(p, qt, kt)) {
+          ++nq[qt];
+          ++nk[kt];
+        }
+    std::vector<int> oq(p.n_tiles), ok(p.n_tiles);
+    for (int t = 0; t < p.n_tiles; ++t) oq[t] = ok[t] = t;
+    std::stable_sort(oq.begin(), oq.end(), [&](int x, int y) { return nq[x] > nq[y]; });
+    std::stable_sort(ok.begin(), ok.end(), [&](int x, int y) { return nk[x] > nk[y]; });
+    for (int t = 0; t < p.n_tiles; ++t) {
+      p.order_q[t] = static_cast<uint16_t>(oq[t]);
+      p.order_k[t] = static_cast<uint16_t>(ok[t]);
+    }
+  }
   const unsigned grid = static_cast<unsigned>(a.B * a.H * p.n_tiles);
   bwd_dq_kernel<<<grid, BTHREADS, DQ_SMEM_BYTES, stream>>>(p);
   cudaError_t e = cudaGetLastError();
