@@ -953,40 +953,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             break;
           }
           __threadfence();
-          // merge the other pieces into this piece's O in TMEM, one piece per
-          // round trip (its (m, l) and whole row loaded together), rescaling
-          // online: O <- O * 2^(M - M') + O_k * 2^(m_k - M')
-          float M = m_run, Lsum = l_run;
+          // Every piece's weight and sum in CTA order, with this piece's own (m, l) in
+          // its place, then the output 32 columns at a time as the sum over the pieces
+          // in that order: the result does not depend on which piece arrived last.  A
+          // row without visible keys in a piece adds nothing.
+          auto ml_of = [&](int k) -> float2 {
+            if (k == me) return make_float2(m_run, l_run);
+            return __ldcg(reinterpret_cast<const float2*>(
+                       p.ws + static_cast<size_t>(slot_of(k)) * PART_FLOATS +
+                       static_cast<size_t>(ROWS) * HEAD_DIM) + row_l);
+          };
+          float M = -INFINITY;
+          for (int k = 0; k < np; ++k) M = fmaxf(M, ml_of(k).x);
+          float Lsum = 0.f;
           for (int k = 0; k < np; ++k) {
-            if (k == me) continue;
-            const float* src = p.ws + static_cast<size_t>(slot_of(k)) * PART_FLOATS;
-            const float2 mk = __ldcg(reinterpret_cast<const float2*>(src + static_cast<size_t>(ROWS) * HEAD_DIM) + row_l);
-            float4 o[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __ldcg(reinterpret_cast<const float4*>(src) + j * ROWS + row_l);
-            // a row without visible keys in piece k leaves the row unchanged; the
-            // TMEM accesses below stay warp-uniform either way
-            const bool none = (mk.x == -INFINITY);
-            const float Mn = none ? M : fmaxf(M, mk.x);
-            const float a = none ? 1.f : ((M == -INFINITY) ? 0.f : ex2(M - Mn));
-            const float bk = none ? 0.f : ex2(mk.x - Mn);
-            Lsum = Lsum * a + mk.y * bk;
-            M = Mn;
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {
-              uint32_t v[32];
-              tmem_ld32(tO + g * 32, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                v[4 * j] = __float_as_uint(__uint_as_float(v[4 * j]) * a + o[g * 8 + j].x * bk);
-                v[4 * j + 1] = __float_as_uint(__uint_as_float(v[4 * j + 1]) * a + o[g * 8 + j].y * bk);
-                v[4 * j + 2] = __float_as_uint(__uint_as_float(v[4 * j + 2]) * a + o[g * 8 + j].z * bk);
-                v[4 * j + 3] = __float_as_uint(__uint_as_float(v[4 * j + 3]) * a + o[g * 8 + j].w * bk);
-              }
-              tmem_st32(tO + g * 32, v);
-            }
-            tmem_wait_st();
+            const float2 mk = ml_of(k);
+            Lsum += (mk.x == -INFINITY) ? 0.f : mk.y * ex2(mk.x - M);
           }
           const float invL = 1.f / Lsum;
           if (p.lse && s_tok < p.sched.Sq) {
@@ -995,9 +977,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
 #pragma unroll 1
           for (int g = 0; g < 4; ++g) {  // 32 output columns per pass
-            uint32_t v[32];
-            tmem_ld32(tO + g * 32, v);
-            tmem_wait_ld();
+            float acc[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) acc[j] = 0.f;
+            for (int k = 0; k < np; ++k) {
+              const float mk = ml_of(k).x;
+              const float sk = (mk == -INFINITY) ? 0.f : ex2(mk - M);
+              if (k == me) {
+                uint32_t v[32];
+                tmem_ld32(tO + g * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) acc[j] += __uint_as_float(v[j]) * sk;
+              } else {
+                const float4* src = reinterpret_cast<const float4*>(
+                    p.ws + static_cast<size_t>(slot_of(k)) * PART_FLOATS);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float4 o = __ldcg(src + (g * 8 + j) * ROWS + row_l);
+                  acc[4 * j] += o.x * sk;
+                  acc[4 * j + 1] += o.y * sk;
+                  acc[4 * j + 2] += o.z * sk;
+                  acc[4 * j + 3] += o.w * sk;
+                }
+              }
+            }
             if (g == 3) {
               tc_fence_before();
               mbar_arrive(&bar[B_O_FREE + q]);
@@ -1006,11 +1010,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint4* xrow = reinterpret_cast<uint4*>(xp + lane * XPOSE_PITCH);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              xrow[j] = make_uint4(
-                  pack_bf16x2(__uint_as_float(v[8 * j]) * invL, __uint_as_float(v[8 * j + 1]) * invL),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 2]) * invL, __uint_as_float(v[8 * j + 3]) * invL),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 4]) * invL, __uint_as_float(v[8 * j + 5]) * invL),
-                  pack_bf16x2(__uint_as_float(v[8 * j + 6]) * invL, __uint_as_float(v[8 * j + 7]) * invL));
+              xrow[j] = make_uint4(pack_bf16x2(acc[8 * j] * invL, acc[8 * j + 1] * invL),
+                                   pack_bf16x2(acc[8 * j + 2] * invL, acc[8 * j + 3] * invL),
+                                   pack_bf16x2(acc[8 * j + 4] * invL, acc[8 * j + 5] * invL),
+                                   pack_bf16x2(acc[8 * j + 6] * invL, acc[8 * j + 7] * invL));
             __syncwarp();
 #pragma unroll
             for (int k = 0; k < 4; ++k) {

@@ -270,15 +270,32 @@ def test_single_visible_key_exact():
     assert np.array_equal(got[:, 0], O.widen_bf16(v)[:, 0])
 
 
-@pytest.mark.parametrize("wi", [1, 0])
+@pytest.mark.parametrize("wi", [1, 0, 2])
 def test_repeatable_bitwise(wi):
-    """Identical calls give identical bytes (the split combine sums pieces in a fixed order)."""
+    """Identical calls give identical bytes.  Workload 2 splits units across CTAs: the
+    combine sums the pieces in CTA order whichever piece arrives last."""
     w = WORKLOADS[wi]
     inp = synth.make_inputs(w, 11)
     args = (inp["q"], inp["k"], inp["v"], inp.get("cache_k"), inp.get("cache_v"), w.cache_tokens)
     first = run_forward(w.layout, w.heads, *args)
-    for _ in range(4):
+    for _ in range(6):
         assert np.array_equal(run_forward(w.layout, w.heads, *args), first)
+
+
+def test_repeatable_bitwise_many_pieces():
+    """Two heads over a long cache: each unit is cut into many pieces (split combine)."""
+    lay = L_(MODE_DECODE, 1, 1, 4, 8, 4, 40)
+    heads, cache_len = 2, 40 * 36
+    rng = np.random.default_rng(77)
+    q = rand_bits(rng, (1, lay.q_len, heads, D))
+    k = rand_bits(rng, (1, lay.self_kv_len, heads, D))
+    v = rand_bits(rng, (1, lay.self_kv_len, heads, D))
+    ck = rand_bits(rng, (1, cache_len, heads, D))
+    cv = rand_bits(rng, (1, cache_len, heads, D))
+    first = run_forward(lay, heads, q, k, v, ck, cv, cache_len)
+    assert_close(first, oracle_full(lay, q, k, v, ck, cv, cache_len), "many pieces")
+    for _ in range(6):
+        assert np.array_equal(run_forward(lay, heads, q, k, v, ck, cv, cache_len), first)
 
 
 def test_decode_matches_prefill_last_chunk():
