@@ -163,7 +163,7 @@ def test_e4m3_attention_elementwise(name, lay, heads, cache_len):
     assert_close(got, oracle_e4m3(lay, q8, k8, v, ck8, cv, cache_len), "e4m3 " + name)
 
 
-@pytest.mark.parametrize("wi", [1, 3, 5])
+@pytest.mark.parametrize("wi", [1, 2, 3, 5])
 def test_e4m3_workload_full_elementwise(wi):
     w = WORKLOADS[wi]
     lay = w.layout
