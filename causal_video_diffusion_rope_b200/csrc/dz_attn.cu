@@ -975,8 +975,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const long long li = (static_cast<long long>(b) * p.H + h) * p.sched.Sq + s_tok;
             if (in_bounds(li, p.out_elems / HEAD_DIM, p.status)) p.lse[li] = M + __log2f(Lsum);
           }
+          // the first other piece's next 32 columns are loaded while this pass runs
+          const int kp = me == 0 ? 1 : 0;
+          const float4* srcp = reinterpret_cast<const float4*>(p.ws + static_cast<size_t>(slot_of(kp)) * PART_FLOATS);
+          float4 nxt[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) nxt[j] = __ldcg(srcp + j * ROWS + row_l);
 #pragma unroll 1
           for (int g = 0; g < 4; ++g) {  // 32 output columns per pass
+            float4 cur[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
+            if (g < 3) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) nxt[j] = __ldcg(srcp + ((g + 1) * 8 + j) * ROWS + row_l);
+            }
             float acc[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) acc[j] = 0.f;
@@ -989,6 +1002,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) acc[j] += __uint_as_float(v[j]) * sk;
+              } else if (k == kp) {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  acc[4 * j] += cur[j].x * sk;
+                  acc[4 * j + 1] += cur[j].y * sk;
+                  acc[4 * j + 2] += cur[j].z * sk;
+                  acc[4 * j + 3] += cur[j].w * sk;
+                }
               } else {
                 const float4* src = reinterpret_cast<const float4*>(
                     p.ws + static_cast<size_t>(slot_of(k)) * PART_FLOATS);
