@@ -706,6 +706,34 @@ def run_e4m3(args, rank: int, world: int, local_rank: int, config: dict):
                         e2e_call, max(3, min(args.steps, 200)), world)
     e2e["value"] = round(job_throughput(fl, e2e.pop("steps_done"), world, e2e.pop("ms")), 3)
     n_sets, set_bytes = st.n_sets, st.set_bytes
+    # a decode call from bf16 q and k: rotation and quantisation of q and the chunk's k
+    # in one pass each (dz_rope3d_e4m3), then the attention on the E4M3 cache
+    whole = None
+    lay = w.layout
+    if lay.mode == synth.MODE_DECODE:
+        B, H, D = lay.batch, w.heads, w.head_dim
+        rng = np.random.default_rng(5000 + rank)
+        bf = [{x: torch.from_numpy(synth.normal_bf16(rng, (B, lay.q_len, H, D)).view(np.int16))
+               .to(dev).view(torch.bfloat16) for x in ("q", "k")} for _ in range(n_sets)]
+        q8b = torch.empty((B, lay.q_len, H, D), dtype=torch.uint8, device=dev)
+        k8b = torch.empty_like(q8b)
+
+        def whole_call(i):
+            b = bf[i % n_sets]
+            st.dz.dz_rope3d_e4m3(st.h, b["q"], q8b, B, lay.q_len, st.dl, lay.num_chunks,
+                                 synth.E4M3_Q_SCALE, stream)
+            st.dz.dz_rope3d_e4m3(st.h, b["k"], k8b, B, lay.q_len, st.dl, lay.num_chunks,
+                                 synth.E4M3_K_SCALE, stream)
+            st.call(i, stream, q8=q8b, k8=k8b)
+
+        nw = max(20, min(args.steps, 2400))
+        wms, _ = time_graph(stream, whole_call, nw, 3, world, dev)
+        st.dz.dz_attn_sync_status(st.h, stream)
+        wus = 1e3 * wms / nw
+        whole = {"what": "dz_rope3d_e4m3 of q and of the chunk's k, then the E4M3 attention",
+                 "us_per_call": round(wus, 3), "tflops": round(fl / (wus * 1e-6) / 1e12, 2),
+                 "launches_per_call": 3}
+        del bf, q8b, k8b
     # the quantisation that feeds the variant (dz_quantize_e4m3), HBM-bound: 64 Mi bf16
     # values (128 MiB read, 64 MiB written) per call, two buffers alternating
     nq = 64 << 20
@@ -733,6 +761,8 @@ def run_e4m3(args, rank: int, world: int, local_rank: int, config: dict):
             "dtype": "e4m3 q/k, bf16 v/p/out, fp32 accumulation",
             "data": "synthetic (E4M3 codes of N(0,1) q, k; N(0,1) bf16 v)",
             "config": dict(config, op="attention_e4m3", q_scale=synth.E4M3_Q_SCALE,
+                           rope="q and k arrive rotated as E4M3 codes (call_from_bf16: rotated "
+                                "and quantised by dz_rope3d_e4m3 inside the timed call)",
                            k_scale=synth.E4M3_K_SCALE,
                            l2=f"inputs cycle through {n_sets} sets "
                               f"({n_sets * set_bytes / 2**20:.0f} MiB > 126 MB L2)",
@@ -745,7 +775,7 @@ def run_e4m3(args, rank: int, world: int, local_rank: int, config: dict):
                          "frac_of_bf16_peak": round(tf / peak_tf, 4),
                          "kernel": "chunk_attn_kernel (E4M3 instantiation)",
                          "kernel_us": round(ms_per_step * 1e3, 3)},
-            "quantize": quant,
+            "quantize": quant, "call_from_bf16": whole,
             "cpu_baseline": None, "e2e": e2e, "gpu_launches": args.steps, "clocks": clocks}
     print(json.dumps(line), flush=True)
 

@@ -379,8 +379,9 @@ dz_status dz_attn_destroy(dz_attn_t a) {
   return cuda_status(e);
 }
 
-dz_status dz_rope3d(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
-                    const dz_chunk_layout* layout, int32_t first_chunk, void* stream) {
+static dz_status rope3d_call(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
+                             const dz_chunk_layout* layout, int32_t first_chunk, float e4m3_scale,
+                             void* stream) {
   if (!a || !x || !y || !layout || B < 1 || S < 0 || first_chunk < 0) return DZ_ERR_INVALID_ARG;
   dz_chunk_layout l = *layout;
   l.batch = B;
@@ -393,8 +394,22 @@ dz_status dz_rope3d(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
   st = check_positions(a, g, first_chunk, first_chunk + (S - 1) / g.L);
   if (st != DZ_OK) return st;
   return cuda_status(dz::launch_rope3d(x, y, B, S, a->desc.num_heads, g, first_chunk,
-                                       tables_of(a), a->status, static_cast<cudaStream_t>(stream)),
+                                       tables_of(a), a->status, static_cast<cudaStream_t>(stream),
+                                       nullptr, nullptr, 0, e4m3_scale),
                      "rope3d launch");
+}
+
+dz_status dz_rope3d(dz_attn_t a, const void* x, void* y, int32_t B, int32_t S,
+                    const dz_chunk_layout* layout, int32_t first_chunk, void* stream) {
+  return rope3d_call(a, x, y, B, S, layout, first_chunk, 0.f, stream);
+}
+
+dz_status dz_rope3d_e4m3(dz_attn_t a, const void* x, void* y8, int32_t B, int32_t S,
+                         const dz_chunk_layout* layout, int32_t first_chunk, float scale,
+                         void* stream) {
+  if (!(scale > 0.f) || !std::isfinite(scale)) return DZ_ERR_INVALID_ARG;
+  if (x == y8 && x != nullptr) return DZ_ERR_INVALID_ARG;  // one byte per element: no in-place
+  return rope3d_call(a, x, y8, B, S, layout, first_chunk, scale, stream);
 }
 
 // The attention call; with lse != null (training form) it also writes each query

@@ -183,11 +183,14 @@ cudaError_t launch_fill_i32(int* x, size_t n, int value, cudaStream_t stream);
 #endif
 
 // Rotates x into y (and x1 into y1 when x1 is not null) for B x S tokens; with
-// period > 0 token s is rotated at the position of token s % period.  `status`
-// receives the bounds-checked build's index faults.
+// period > 0 token s is rotated at the position of token s % period.  With
+// e4m3_scale > 0 the outputs are the E4M3 codes of the rotated bf16 values times
+// e4m3_scale (one byte per element).  `status` receives the bounds-checked build's
+// index faults.
 cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const ChunkGeom& g,
                           int first_chunk, const RopeTables& r, int* status, cudaStream_t stream,
-                          const void* x1 = nullptr, void* y1 = nullptr, int period = 0);
+                          const void* x1 = nullptr, void* y1 = nullptr, int period = 0,
+                          float e4m3_scale = 0.f);
 
 // y[0:n] = E4M3 codes of x[0:n] * scale (round to nearest even, saturating at 448).
 cudaError_t launch_quantize_e4m3(const __nv_bfloat16* x, uint8_t* y, long long n, float scale,

@@ -71,15 +71,30 @@ cudaError_t launch_kv_copy(const void* k, const void* v, void* ck, void* cv, int
 // token s % period (the noisy half of a teacher-forcing sequence shares the
 // clean half's positions).
 // x and y may be the same buffer (in place): each thread reads and then writes
-// the same 16 bytes, so they are not declared __restrict__.
+// the same 16 bytes, so they are not declared __restrict__.  With E4M3 output each
+// rotated bf16 value is also quantised (times `scale`, as dz_quantize_e4m3 does) and
+// a 16-byte chunk becomes 8 bytes.
 // ---------------------------------------------------------------------------
 constexpr int ROPE_BLOCK = 128;
 constexpr int ROPE_UNROLL = 8;  // chunks per thread per pass: 64 heads with 128 threads
 
-__global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, uint4* y0,
-                                                            const uint4* x1, uint4* y1, int S,
+// Four bf16 values (two packed pairs) times scale, as E4M3 codes: the fp32 product,
+// rounded to nearest even with magnitudes past 448 saturating.
+__device__ __forceinline__ uint32_t e4m3x4(uint32_t lo2, uint32_t hi2, float scale) {
+  const float2 a = make_float2(__fmul_rn(__uint_as_float(lo2 << 16), scale),
+                               __fmul_rn(__uint_as_float(lo2 & 0xffff0000u), scale));
+  const float2 b = make_float2(__fmul_rn(__uint_as_float(hi2 << 16), scale),
+                               __fmul_rn(__uint_as_float(hi2 & 0xffff0000u), scale));
+  const uint32_t pa = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
+  const uint32_t pb = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
+  return pa | (pb << 16);
+}
+
+template <bool E4M3>
+__global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, void* y0,
+                                                            const uint4* x1, void* y1, int S,
                                                             int H, ChunkGeom g, int first_chunk,
-                                                            int period, RopeTables r,
+                                                            int period, RopeTables r, float scale,
                                                             int* status) {
   const long long token = blockIdx.x;  // b * S + s
   int s = static_cast<int>(token % S);
@@ -88,7 +103,7 @@ __global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, uin
   token_pos(g, s, first_chunk, t, hh, w);
   const int nvec = H * (HEAD_DIM / 8);
   const uint4* src = (blockIdx.y == 0 ? x0 : x1) + token * nvec;
-  uint4* dst = (blockIdx.y == 0 ? y0 : y1) + token * nvec;
+  void* dst_base = blockIdx.y == 0 ? y0 : y1;
   const int j0 = (threadIdx.x & 15) * 4;  // ROPE_BLOCK is a multiple of 16
   float2 cs[4];
 #pragma unroll
@@ -103,22 +118,33 @@ __global__ void __launch_bounds__(ROPE_BLOCK) rope3d_kernel(const uint4* x0, uin
 #pragma unroll
     for (int u = 0; u < ROPE_UNROLL; ++u) {
       const int i = i0 + u * ROPE_BLOCK;
-      if (i < nvec)
-        dst[i] = make_uint4(rope_pair(v[u].x, cs[0]), rope_pair(v[u].y, cs[1]),
-                            rope_pair(v[u].z, cs[2]), rope_pair(v[u].w, cs[3]));
+      if (i < nvec) {
+        const uint4 o = make_uint4(rope_pair(v[u].x, cs[0]), rope_pair(v[u].y, cs[1]),
+                                   rope_pair(v[u].z, cs[2]), rope_pair(v[u].w, cs[3]));
+        if constexpr (E4M3)
+          (static_cast<uint2*>(dst_base) + token * nvec)[i] =
+              make_uint2(e4m3x4(o.x, o.y, scale), e4m3x4(o.z, o.w, scale));
+        else
+          (static_cast<uint4*>(dst_base) + token * nvec)[i] = o;
+      }
     }
   }
 }
 
 cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const ChunkGeom& g,
                           int first_chunk, const RopeTables& r, int* status, cudaStream_t stream,
-                          const void* x1, void* y1, int period) {
+                          const void* x1, void* y1, int period, float e4m3_scale) {
   const long long tokens = static_cast<long long>(B) * S;
   if (tokens <= 0) return cudaSuccess;
   dim3 grid(static_cast<unsigned>(tokens), x1 ? 2 : 1);
-  rope3d_kernel<<<grid, ROPE_BLOCK, 0, stream>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y),
-                                          static_cast<const uint4*>(x1), static_cast<uint4*>(y1),
-                                          S, H, g, first_chunk, period, r, status);
+  if (e4m3_scale > 0.f)
+    rope3d_kernel<true><<<grid, ROPE_BLOCK, 0, stream>>>(static_cast<const uint4*>(x), y,
+                                                         static_cast<const uint4*>(x1), y1, S, H, g,
+                                                         first_chunk, period, r, e4m3_scale, status);
+  else
+    rope3d_kernel<false><<<grid, ROPE_BLOCK, 0, stream>>>(static_cast<const uint4*>(x), y,
+                                                          static_cast<const uint4*>(x1), y1, S, H, g,
+                                                          first_chunk, period, r, 0.f, status);
   return cudaGetLastError();
 }
 
@@ -128,16 +154,6 @@ cudaError_t launch_rope3d(const void* x, void* y, int B, int S, int H, const Chu
 // thread turns 16 bf16 values (two 16-byte loads) into one 16-byte store; the last
 // n % 16 elements go one per thread.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t e4m3x4(uint32_t lo2, uint32_t hi2, float scale) {
-  const float2 a = make_float2(__fmul_rn(__uint_as_float(lo2 << 16), scale),
-                               __fmul_rn(__uint_as_float(lo2 & 0xffff0000u), scale));
-  const float2 b = make_float2(__fmul_rn(__uint_as_float(hi2 << 16), scale),
-                               __fmul_rn(__uint_as_float(hi2 & 0xffff0000u), scale));
-  const uint32_t pa = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
-  const uint32_t pb = __nv_cvt_float2_to_fp8x2(b, __NV_SATFINITE, __NV_E4M3);
-  return pa | (pb << 16);
-}
-
 __global__ void __launch_bounds__(256) quantize_e4m3_kernel(const uint4* __restrict__ x,
                                                             uint4* __restrict__ y, long long nvec,
                                                             float scale) {

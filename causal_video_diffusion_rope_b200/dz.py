@@ -37,6 +37,7 @@ EXPORTS = [
     "dz_kvcache_append", "dz_kvcache_replace", "dz_attn_sync_status", "dz_status_string",
     "dz_chunk_attn_forward_noalloc", "dz_qkv_rope", "dz_chunk_attn_forward_lse",
     "dz_chunk_attn_backward", "dz_chunk_attn_forward_e4m3", "dz_quantize_e4m3",
+    "dz_rope3d_e4m3",
 ]
 
 
@@ -102,6 +103,8 @@ def bind(lib: ctypes.CDLL) -> ctypes.CDLL:
                                                ctypes.POINTER(dz_chunk_layout), ctypes.c_float,
                                                ctypes.c_float, vp, vp]
     lib.dz_quantize_e4m3.argtypes = [vp, vp, vp, ctypes.c_int64, ctypes.c_float, vp]
+    lib.dz_rope3d_e4m3.argtypes = [vp, vp, vp, i32, i32, ctypes.POINTER(dz_chunk_layout), i32,
+                                   ctypes.c_float, vp]
     lib.dz_attn_sync_status.argtypes = [vp, vp]
     lib.dz_status_string.argtypes = [ctypes.c_int]
     lib.dz_status_string.restype = ctypes.c_char_p
@@ -209,6 +212,12 @@ def dz_chunk_attn_forward_e4m3(handle: int, q8, k8, v, cache: Optional[dz_kvcach
                                              ctypes.byref(layout), q_scale, k_scale, _ptr(out),
                                              _stream(stream)),
            "dz_chunk_attn_forward_e4m3")
+
+
+def dz_rope3d_e4m3(handle: int, x, y8, B: int, S: int, layout: dz_chunk_layout, first_chunk: int,
+                   scale: float, stream=None) -> None:
+    _check(load().dz_rope3d_e4m3(handle, _ptr(x), _ptr(y8), B, S, ctypes.byref(layout), first_chunk,
+                                 scale, _stream(stream)), "dz_rope3d_e4m3")
 
 
 def dz_quantize_e4m3(handle: int, x, y, n: int, scale: float, stream=None) -> None:

@@ -209,6 +209,15 @@ dz_status dz_chunk_attn_forward_e4m3(dz_attn_t handle, const void* q8, const voi
                                      const dz_chunk_layout* layout, float q_scale, float k_scale,
                                      void* out, void* stream);
 
+/* dz_rope3d followed by dz_quantize_e4m3 in one pass: y8 receives the E4M3 codes of
+ * the rotated bf16 values times `scale`, the same bytes the two calls give.  x bf16
+ * [B][S][H][128], y8 uint8 [B][S][H][128], both 16-byte aligned, no overlap.
+ * Errors: as dz_rope3d, and DZ_ERR_INVALID_ARG for a scale that is not finite and
+ * positive or y8 == x. */
+dz_status dz_rope3d_e4m3(dz_attn_t handle, const void* x, void* y8, int32_t B, int32_t S,
+                         const dz_chunk_layout* layout, int32_t first_chunk, float scale,
+                         void* stream);
+
 /* E4M3 quantisation of n bf16 values: y[i] = E4M3(float(x[i]) * scale), the
  * product formed in fp32 and rounded to the nearest E4M3 value (ties to even),
  * magnitudes past 448 saturating to 448, sign kept (-0 for negatives that round

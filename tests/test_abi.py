@@ -86,6 +86,8 @@ def test_calls_reject_null_handle(lib):
     assert lib.dz_chunk_attn_forward_e4m3(None, 16, 16, 16, None, ctypes.byref(lay), 64.0, 16.0,
                                           16, None) == dz.DZ_ERR_INVALID_ARG
     assert lib.dz_quantize_e4m3(None, 16, 16, 128, 1.0, None) == dz.DZ_ERR_INVALID_ARG
+    assert lib.dz_rope3d_e4m3(None, 16, 32, 1, 1, ctypes.byref(lay), 0, 1.0, None) == \
+        dz.DZ_ERR_INVALID_ARG
     # a null layout or output pointer is rejected before any handle lookup
     assert lib.dz_chunk_attn_forward_lse(None, 16, 16, 16, None, 16, 16, None) == \
         dz.DZ_ERR_INVALID_ARG

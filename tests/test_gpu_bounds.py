@@ -47,9 +47,11 @@ def cases(fn):
 @pytest.fixture(scope="module")
 def checked():
     """The dz binding routed to the bounds-checked library for this module's tests."""
+    import test_gpu_e4m3 as E
     import test_gpu_parity as P
     product = dz.load()
     P.teardown_module(P)  # handles of the product library, if any are cached
+    E.teardown_module(E)
     lib = dz.bind(ctypes.CDLL(build.TEST_LIB))
     lib.dz_test_shrink_out.argtypes = [ctypes.c_int64]
     lib.dz_test_shrink_out.restype = None
@@ -62,6 +64,7 @@ def checked():
     finally:
         lib.dz_test_shrink_out(0)
         P.teardown_module(P)  # handles made with the checked library
+        E.teardown_module(E)
         dz._lib = product
 
 
@@ -102,6 +105,14 @@ def test_projection_in_bounds(checked):
 def test_backward_in_bounds(checked):
     import test_gpu_bwd as B
     run_all(B.test_backward_small, checked)
+
+
+def test_e4m3_in_bounds(checked):
+    import test_gpu_e4m3 as E
+    run_all(E.test_e4m3_attention_elementwise, checked)
+    E.test_e4m3_workload_full_elementwise(1)
+    E.test_e4m3_workload_full_elementwise(3)
+    assert checked.dz_test_bounds_faults() == 0, "e4m3 workloads: index fault"
 
 
 def test_planted_extent_fault_is_reported(checked):

@@ -9,8 +9,11 @@
   (fp32 accumulation of the E4M3 products, P to bf16, fp32 PV accumulation, bf16
   output) -- the bf16 path's bounds apply unchanged: max |gpu - ref| <= 2e-2 and
   rel-L2 <= 5e-3 per call.
-* The quantisation's own effect (rotation by dz_rope3d, E4M3 by dz_quantize_e4m3,
-  then the FP8 attention, against the oracle on the unquantised bf16 operands):
+* dz_rope3d_e4m3: the bytes of dz_rope3d followed by dz_quantize_e4m3, and the
+  oracle's codes of its own rotation rounded to bf16 except at bf16 rounding
+  boundaries (neighbouring codes there).
+* The quantisation's own effect (rotation and E4M3 by dz_rope3d_e4m3, then the FP8
+  attention, against the oracle on the unquantised bf16 operands):
   E4M3 keeps 3 mantissa bits, so each operand carries a relative rounding error of
   rms eps (about 2.7% for normally distributed values, at most 2^-4); a score
   q.k/sqrt(128) over independent normal entries then moves by about sqrt(2) * eps of
@@ -103,6 +106,56 @@ def test_quantize_argument_errors():
     dz.dz_quantize_e4m3(h, x, y, 0, 1.0)  # empty: nothing to do
 
 
+# ------------------------------------------------------------------ rotation + quantisation in one pass
+
+@pytest.mark.parametrize("B,S,H,F,gh,gw,na,t0,first,scale", [
+    (1, 108, 2, 1, 4, 8, 4, 0, 0, 64.0),
+    (1, 464, 40, 2, 11, 20, 24, 0, 4, 16.0),
+    (2, 928, 3, 2, 11, 20, 24, 5, 31, 57.3),
+    (1, 37, 1, 1, 1, 1, 0, 100, 0, 1.0 / 8),
+])
+def test_rope3d_e4m3(B, S, H, F, gh, gw, na, t0, first, scale):
+    """dz_rope3d_e4m3 gives the bytes of dz_rope3d followed by dz_quantize_e4m3, and the
+    oracle's codes of its own rotation rounded to bf16 (nearest even) everywhere except
+    where that rotation lies within fp32 rounding of a bf16 rounding boundary: there the
+    two codes may be neighbours."""
+    from gpu_util import bf16_round
+    rng = np.random.default_rng(11 + S)
+    x = synth.bf16_bits_from_f32(rng.standard_normal((B, S, H, D)).astype(np.float32) * 2.0)
+    h = handle(H)
+    lay = dz.make_layout(0, B, F, gh, gw, na, 0, t0)
+    xd = to_dev(x)
+    y8 = torch.full((B, S, H, D), 0xAA, dtype=torch.uint8, device="cuda")
+    dz.dz_rope3d_e4m3(h, xd, y8, B, S, lay, first, scale)
+    y16 = torch.empty_like(xd)
+    dz.dz_rope3d(h, xd, y16, B, S, lay, first)
+    q8 = torch.empty_like(y8)
+    dz.dz_quantize_e4m3(h, y16, q8, q8.numel(), scale)
+    dz.dz_attn_sync_status(h)
+    got = y8.cpu().numpy()
+    assert np.array_equal(got, q8.cpu().numpy()), "fused pass differs from the two calls"
+    ref = O.quantize_e4m3(bf16_round(O.rope3d(O.widen_bf16(x), F, gh, gw, na, t0, first))
+                          .astype(np.float32), scale)
+    bad = np.nonzero(got != ref)
+    assert bad[0].size <= max(2, got.size // 100000), bad[0].size
+    g, r = got[bad].astype(np.int64), ref[bad].astype(np.int64)
+    assert np.all((g & 0x80) == (r & 0x80)) and np.all(np.abs((g & 0x7F) - (r & 0x7F)) <= 1)
+
+
+def test_rope3d_e4m3_argument_errors():
+    h = handle(2)
+    lay = dz.make_layout(0, 1, 1, 4, 8, 4, 0, 0)
+    x = torch.zeros((1, 36, 2, D), dtype=torch.bfloat16, device="cuda")
+    y = torch.zeros((1, 36, 2, D), dtype=torch.uint8, device="cuda")
+    for bad in (0.0, -2.0, float("nan")):
+        with pytest.raises(dz.DzError) as e:
+            dz.dz_rope3d_e4m3(h, x, y, 1, 36, lay, 0, bad)
+        assert e.value.status == dz.DZ_ERR_INVALID_ARG
+    with pytest.raises(dz.DzError) as e:
+        dz.dz_rope3d_e4m3(h, x, x, 1, 36, lay, 0, 1.0)
+    assert e.value.status == dz.DZ_ERR_INVALID_ARG
+
+
 # ------------------------------------------------------------------ attention on E4M3 q, k
 
 def run_e4m3(lay: Layout, heads: int, q8, k8, v, cache_k8=None, cache_v=None, cache_len=0):
@@ -188,24 +241,22 @@ def test_e4m3_argument_errors():
 
 
 def test_e4m3_pipeline_quantisation_error():
-    """Workload 1 through the FP8 path from bf16 q, k, v: dz_rope3d, dz_quantize_e4m3,
-    then the E4M3 attention, against the oracle on the unquantised operands."""
+    """Workload 1 through the FP8 path from bf16 q, k, v: dz_rope3d_e4m3 (rotation and
+    quantisation in one pass) for q and the chunk's k, dz_quantize_e4m3 for the cached
+    (already rotated) keys, then the E4M3 attention, against the oracle on the
+    unquantised operands."""
     w = WORKLOADS[1]
     lay = w.layout
     B, H, L = lay.batch, w.heads, lay.chunk_len
     inp = synth.make_inputs(w, 11)
     h = handle(H)
     dl = dz.layout_from(lay)
-    qr = torch.empty((B, L, H, D), dtype=torch.bfloat16, device="cuda")
-    kr = torch.empty_like(qr)
-    dz.dz_rope3d(h, to_dev(inp["q"]), qr, B, L, dl, lay.num_chunks)
-    dz.dz_rope3d(h, to_dev(inp["k"]), kr, B, L, dl, lay.num_chunks)
     q8 = torch.empty((B, L, H, D), dtype=torch.uint8, device="cuda")
     k8 = torch.empty_like(q8)
     cap = w.cache_tokens
     ck8 = torch.empty((B, cap, H, D), dtype=torch.uint8, device="cuda")
-    dz.dz_quantize_e4m3(h, qr, q8, q8.numel(), QS)
-    dz.dz_quantize_e4m3(h, kr, k8, k8.numel(), KS)
+    dz.dz_rope3d_e4m3(h, to_dev(inp["q"]), q8, B, L, dl, lay.num_chunks, QS)
+    dz.dz_rope3d_e4m3(h, to_dev(inp["k"]), k8, B, L, dl, lay.num_chunks, KS)
     dz.dz_quantize_e4m3(h, to_dev(inp["cache_k"]), ck8, ck8.numel(), KS)
     cv = to_dev(inp["cache_v"])
     cache = dz.make_cache(ck8, cv, B, cap, w.cache_tokens, L)
