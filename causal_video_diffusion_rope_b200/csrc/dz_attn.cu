@@ -37,8 +37,9 @@
 // share a few heads' keys through L2, and split only the remaining units.  A unit that one
 // CTA covers entirely writes bf16 output directly; otherwise each piece counts
 // its arrival on the unit's counter, every piece but the last to arrive
-// publishes fp32 partial (O, m, l) to the workspace, and the last one merges
-// them into its own O in TMEM.  With the call's q and own k rotated once into a
+// publishes fp32 partial (O, m, l) to the workspace, and the last one sums all
+// pieces in CTA order (its own O read from TMEM in its place), so the result does
+// not depend on the arrival order.  With the call's q and own k rotated once into a
 // workspace beforehand (or given rotated), the rotary gate only passes tiles on.
 //
 // E4M3 variant (second template argument): q and k arrive rotated as E4M3 codes (one
