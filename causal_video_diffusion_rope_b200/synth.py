@@ -3,7 +3,9 @@
 This module holds shapes and random draws only: no attention, rotary or mask
 arithmetic lives here.  Every tensor is drawn as float32 standard normals from
 ``numpy.random.default_rng(seed)`` and rounded to bfloat16 (round to nearest,
-ties to even), so the same bytes go to the GPU and to the CPU oracle.
+ties to even), so the same bytes go to the GPU and to the CPU oracle; the FP8
+variant's q and k are the same kind of draws cast to E4M3 codes by torch's
+float8_e4m3fn conversion.
 
 Workloads follow the DreamZero pages (Causal WAN DiT: 40 heads, head_dim 128,
 dim 5120 -- "DreamZero_Architecture", section 5 hyper-parameter table; chunked
